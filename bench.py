@@ -1,0 +1,391 @@
+"""Benchmark of the adaptive block-sparse attention path on B200.
+
+One step = one pass of the whole path over one Wan-like attention layer held in
+HBM: reorder(Q, K, V) -> route -> repair -> block-sparse attention -> inverse
+reorder.  `value` is the step's throughput in actual (sparse) attention TFLOP/s;
+the JSON line also carries the dense-equivalent rate, the routing GB/s, the
+attention kernel's roofline fraction, an end-to-end figure through host buffers,
+the clocks seen while timing, and the CPU oracle timed on a bounded sample.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config wan480p] [--impl reference]
+
+Multi-GPU (torchrun): every rank runs its own replica of the layer (weak scaling,
+no data-path collective); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+DEFAULT_CONFIG = "wan480p"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(synth.CONFIGS))
+    ap.add_argument("--impl", default="fva", choices=["fva", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--static-order", action="store_true", help="item-id order instead of the LPT work list")
+    return ap.parse_args()
+
+
+def workload_desc(cfg) -> dict:
+    return {
+        "workload": f"{cfg.name}: single attention layer, B={cfg.B}, H={cfg.H}, head_dim={cfg.d}, "
+                    f"latent {cfg.T}x{cfg.Y}x{cfg.X}={cfg.N} tokens, tiles {cfg.tt}x{cfg.ty}x{cfg.tx}={cfg.S} "
+                    f"({cfg.Nb} blocks), p={cfg.p}, k={cfg.k}",
+        "B": cfg.B, "H": cfg.H, "head_dim": cfg.d, "tokens": cfg.N, "tile": cfg.S, "blocks": cfg.Nb,
+        "p": cfg.p, "k": cfg.k, "generator": f"random Fourier features sigma={cfg.sigma}, a_h {cfg.a_mode} "
+                                             f"[{cfg.a_lo}, {cfg.a_hi}], noise std {cfg.noise_std:.3g}, seed {cfg.seed}",
+        "l2": f"inputs larger than L2 ({cfg.B * cfg.H * cfg.N * cfg.d * 2 / 1e6:.0f} MB per Q/K/V tensor)",
+    }
+
+
+def load_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "src": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "src": "fallback"}
+
+
+def attn_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("attn.cu", "fva_common.cuh"):
+        h.update(open(os.path.join(ROOT, "block_sparse_attention_44_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:12]
+
+
+def attn_traffic(cfg_name: str, launches_units: float):
+    """DRAM bytes per attention launch from the committed ncu summary, if it was taken on the
+    current attention source; scaled by processed block pairs when captured on a smaller case."""
+    p = os.path.join(ROOT, "profiles", "attn_dram_traffic.md")
+    if not os.path.exists(p):
+        return None
+    txt = open(p).read()
+    m = re.search(r"source_hash:\s*([0-9a-f]+)", txt)
+    b = re.search(r"dram_bytes_per_block_pair:\s*([0-9.eE+]+)", txt)
+    if not m or not b or m.group(1) != attn_source_hash():
+        return None
+    return float(b.group(1)) * launches_units
+
+
+# ------------------------------------------------------------------ clocks ---------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ CPU oracle ---------
+def oracle_sample(cfg, budget_s: float = 10.0):
+    """The oracle, as it stands, on a bounded sample: one head of the workload through the
+    whole path (reorder, route, repair), then masked attention for as many of its query
+    blocks as fit in the time budget.  Returns (TFLOP/s, seconds, description)."""
+    import oracle as O
+    og = O.Geometry.of(cfg.with_(H=1))
+    q, k, v = synth.make_qkv(cfg, heads=[0])
+    t0 = time.perf_counter()
+    qr, kr, vr = (O.reorder(t, og) for t in (q, k, v))
+    rr = O.route(qr, kr, og, cfg.p, cfg.k)
+    rp = O.repair(rr.topp_mask, rr.topk_idx)
+    flops = 0.0
+    n = 0
+    for i in range(og.Nb):
+        O.attention_items(qr, kr, vr, rp.counts, rp.idx, og.S, [(0, 0, i)])
+        flops += 4.0 * og.S * og.S * og.d * float(rp.counts[0, 0, i])
+        n += 1
+        if time.perf_counter() - t0 > budget_s and n >= 4:
+            break
+    dt = time.perf_counter() - t0
+    desc = (f"head 0 of {cfg.name}: reorder+route+repair of the head ({og.Nb} query blocks), then masked "
+            f"float64 attention for {n} of its query blocks; throughput = sparse attention FLOPs executed / "
+            f"wall time of the sample")
+    return flops / dt / 1e12, dt, desc
+
+
+def cpu_cores() -> int:
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        n = max((d.get("num_threads", 1) for d in info), default=1)
+        return int(n)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args, rank: int, world: int):
+    if rank != 0:
+        return
+    cfg = synth.CONFIGS[args.config]
+    vals, secs = [], []
+    desc = ""
+    for s in range(args.warmup + args.steps):
+        v, dt, desc = oracle_sample(cfg, budget_s=3.0)
+        if s >= args.warmup:
+            vals.append(v)
+            secs.append(dt)
+    value = statistics.median(vals)
+    cores = cpu_cores()
+    line = {
+        "impl": "reference", "metric": "block-sparse attention TFLOP/s (actual sparse FLOPs)", "value": value,
+        "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * statistics.median(secs), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": workload_desc(cfg),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ GPU arm ----------
+def run_gpu(args, rank: int, world: int, local_rank: int):
+    import torch
+    import torch.distributed as dist
+    import block_sparse_attention_44_b200 as fva
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    cfg = synth.CONFIGS[args.config]
+    g = fva.Geom.of(cfg)
+    peaks = load_peaks()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, dt, desc = oracle_sample(cfg, budget_s=10.0)
+        cpu = {"value": v, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle", "sample": desc,
+               "seconds": round(dt, 2)}
+
+    q, k, v = synth.make_qkv(cfg)
+    def host_bf16(a):
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
+    qh, kh, vh = (host_bf16(a).pin_memory() for a in (q, k, v))
+    del q, k, v
+    qd, kd, vd = (t.to(dev) for t in (qh, kh, vh))
+    out = torch.empty_like(qd)
+    outh = torch.empty(out.shape, dtype=torch.bfloat16).pin_memory()
+    path = fva.SparseAttention(g, cfg.p, cfg.k, device=dev, use_lpt=not args.static_order)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        path(qd, kd, vd, out, stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    assert fva.fva_get_device_error(stream) == 0
+
+    counts = path.rep.counts
+    pairs = int(counts.sum().item())
+    flops_actual = 4.0 * g.S * g.S * g.d * pairs
+    flops_dense = 4.0 * g.B * g.H * float(g.N) ** 2 * g.d
+    density = pairs / float(g.B * g.H * g.Nb * g.Nb)
+
+    # --- timed region: K whole steps; per-stage events on the launching stream
+    K = args.steps
+    E = lambda: torch.cuda.Event(enable_timing=True)
+    ev = [[E() for _ in range(6)] for _ in range(K)]
+    gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid) if hasattr(
+        torch.cuda.get_device_properties(dev), "uuid") else str(local_rank)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    launches0 = fva.fva_launch_count()
+    with ClockSampler(gpu_id) as clk:
+        start, stop = E(), E()
+        start.record(stream)
+        for s in range(K):
+            e = ev[s]
+            e[0].record(stream)
+            fva.fva_reorder(qd, path.qr, g, stream)
+            fva.fva_reorder(kd, path.kr, g, stream)
+            fva.fva_reorder(vd, path.vr, g, stream)
+            e[1].record(stream)
+            fva.fva_route(path.qr, path.kr, g, cfg.p, cfg.k, path.route.topp_mask, path.route.topk_idx, path.ws,
+                          stream=stream)
+            e[2].record(stream)
+            fva.fva_repair(path.route.topp_mask, path.route.topk_idx, g, cfg.k, path.rep.counts, path.rep.idx,
+                           path.rep.head_work, path.rep.worklist, stream=stream)
+            e[3].record(stream)
+            path.attention(stream)
+            e[4].record(stream)
+            fva.fva_inverse_reorder(path.outr, out, g, stream)
+            e[5].record(stream)
+        stop.record(stream)
+        torch.cuda.synchronize(dev)
+    launches = fva.fva_launch_count() - launches0
+    assert fva.fva_get_device_error(stream) == 0
+    total_ms = start.elapsed_time(stop)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms = total_ms / K
+    stage = np.array([[ev[s][i].elapsed_time(ev[s][i + 1]) for i in range(5)] for s in range(K)])
+    st_mean = stage.mean(axis=0)            # reorder x3, route, repair, attention, inverse (ms)
+    attn_ms = float(st_mean[3])
+    route_ms = float(st_mean[1] + st_mean[2])
+
+    # --- end to end through host buffers (pinned H2D of Q/K/V, the path, D2H of O)
+    h2d = 3 * qh.numel() * 2
+    d2h = outh.numel() * 2
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    s0, s1 = E(), E()
+    s0.record(stream)
+    for _ in range(K):
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        step()
+        outh.copy_(out, non_blocking=True)
+    s1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = s0.elapsed_time(s1) / K
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    if rank != 0:
+        return
+    bytes_route = 2.0 * g.B * g.H * g.N * g.d * 2          # Qr and Kr read once
+    bytes_reorder = 3 * 2.0 * g.B * g.H * g.N * g.d * 2    # Q, K, V read + write
+    achieved = flops_actual / (attn_ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+    traffic = attn_traffic(cfg.name, pairs)
+    value = world * flops_actual / (ms * 1e-3) / 1e12
+    line = {
+        "metric": "block-sparse attention TFLOP/s (actual sparse FLOPs per whole-path step)",
+        "value": value,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": max(args.warmup, 3),
+        "ms_per_step": ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded random-Fourier-feature Q/K, Gaussian V; stands in for Wan2.2 latents)",
+        "config": dict(workload_desc(cfg), parallelism=f"replicas x{world} (no data-path collective)",
+                       order="static" if args.static_order else "lpt"),
+        "dense_equiv_tflops": world * flops_dense / (ms * 1e-3) / 1e12,
+        "attn_kernel_tflops": achieved,
+        "attn_kernel_dense_equiv_tflops": flops_dense / (attn_ms * 1e-3) / 1e12,
+        "density": density,
+        "routing_gbs": bytes_route / (route_ms * 1e-3) / 1e9,
+        "routing_frac_hbm": bytes_route / (route_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+        "reorder_gbs": bytes_reorder / (st_mean[0] * 1e-3) / 1e9,
+        "routing_overhead_pct": 100.0 * route_ms / attn_ms,
+        "stage_ms": {"reorder_qkv": st_mean[0], "route": st_mean[1], "repair": st_mean[2], "attention": st_mean[3],
+                     "inverse_reorder": st_mean[4]},
+        "roofline": {"bound": "tensor", "kernel": "attn_kernel (fva_block_sparse_attn)", "achieved": achieved,
+                     "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "peak_src": f"{peaks['src']} bf16 sustained (kernel timed inside a long step loop)",
+                     "traffic": traffic,
+                     "algorithmic_units": f"{pairs} kept block pairs x {4 * g.S * g.S * g.d} FLOP"},
+        "routing_roofline": {"bound": "hbm", "achieved": bytes_route / (route_ms * 1e-3) / 1e9,
+                             "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                             "frac": bytes_route / (route_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+        "e2e": {"value": world * flops_actual / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": int(launches),
+        "clocks": clk.summary(),
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    import torch
+    import torch.distributed as dist
+    import datetime
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_gpu(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,272 @@
+"""Thin Python binding of libfva.so (the C ABI in include/fva.h).
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels.  PyTorch provides device memory and streams.  Importing fails loudly if
+the library has not been built (``python -m block_sparse_attention_44_b200.build``);
+there is no fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+from typing import Optional
+
+import torch
+
+__all__ = [
+    "FvaError", "Geom", "lib", "fva_reorder", "fva_inverse_reorder", "fva_route_workspace_size", "fva_route",
+    "fva_repair_workspace_size", "fva_repair", "fva_block_sparse_attn", "fva_get_device_error", "fva_last_error",
+    "fva_launch_count", "fva_version", "RouteOutputs", "RepairOutputs", "SparseAttention",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfva.so")
+
+FVA_OK, FVA_ERR_INVALID_ARG, FVA_ERR_UNSUPPORTED, FVA_ERR_CUDA, FVA_ERR_TIMEOUT = range(5)
+_CODES = {1: "FVA_ERR_INVALID_ARG", 2: "FVA_ERR_UNSUPPORTED", 3: "FVA_ERR_CUDA", 4: "FVA_ERR_TIMEOUT"}
+
+
+class FvaError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"{_CODES.get(code, code)}: {msg}")
+        self.code = code
+
+
+class _Geom(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("B", "H", "T", "Y", "X", "d", "tt", "ty", "tx")]
+
+
+@dataclasses.dataclass(frozen=True)
+class Geom:
+    """Batch B, heads H, latent grid T x Y x X, head_dim d, tile tt x ty x tx."""
+
+    B: int
+    H: int
+    T: int
+    Y: int
+    X: int
+    d: int
+    tt: int
+    ty: int
+    tx: int
+
+    @property
+    def N(self) -> int:
+        return self.T * self.Y * self.X
+
+    @property
+    def S(self) -> int:
+        return self.tt * self.ty * self.tx
+
+    @property
+    def Nb(self) -> int:
+        return self.N // self.S
+
+    def c(self) -> _Geom:
+        return _Geom(self.B, self.H, self.T, self.Y, self.X, self.d, self.tt, self.ty, self.tx)
+
+    @staticmethod
+    def of(cfg) -> "Geom":
+        return Geom(cfg.B, cfg.H, cfg.T, cfg.Y, cfg.X, cfg.d, cfg.tt, cfg.ty, cfg.tx)
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m block_sparse_attention_44_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, sz, i32, i64, f32, f64 = (ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32, ctypes.c_int64,
+                                  ctypes.c_float, ctypes.c_double)
+    sig = {
+        "fva_reorder": ([vp, vp, _Geom, vp], ctypes.c_int),
+        "fva_inverse_reorder": ([vp, vp, _Geom, vp], ctypes.c_int),
+        "fva_route_workspace_size": ([_Geom], sz),
+        "fva_route": ([vp, vp, _Geom, f64, i32, vp, vp, vp, vp, sz, vp], ctypes.c_int),
+        "fva_repair_workspace_size": ([_Geom], sz),
+        "fva_repair": ([vp, vp, _Geom, i32, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
+        "fva_block_sparse_attn": ([vp, vp, vp, vp, vp, vp, _Geom, f32, vp, vp], ctypes.c_int),
+        "fva_get_device_error": ([vp, ctypes.POINTER(i32)], ctypes.c_int),
+        "fva_last_error": ([], ctypes.c_char_p),
+        "fva_launch_count": ([], i64),
+        "fva_version": ([], i32),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(L, name)
+        f.argtypes = args
+        f.restype = res
+    return L
+
+
+lib = _load()
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream if torch.cuda.is_available() else None
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _check(rc: int) -> None:
+    if rc != FVA_OK:
+        raise FvaError(rc, lib.fva_last_error().decode())
+
+
+def _need(t: torch.Tensor, dtype: torch.dtype, shape, name: str) -> None:
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name}: must be a CUDA tensor")
+
+
+# ------------------------------------------------------------------ 1:1 wrappers ----
+def fva_reorder(x: torch.Tensor, xr: torch.Tensor, g: Geom, stream=None) -> None:
+    shp = (g.B, g.H, g.N, g.d)
+    _need(x, torch.bfloat16, shp, "x")
+    _need(xr, torch.bfloat16, shp, "xr")
+    _check(lib.fva_reorder(_ptr(x), _ptr(xr), g.c(), _stream(stream)))
+
+
+def fva_inverse_reorder(xr: torch.Tensor, x: torch.Tensor, g: Geom, stream=None) -> None:
+    shp = (g.B, g.H, g.N, g.d)
+    _need(xr, torch.bfloat16, shp, "xr")
+    _need(x, torch.bfloat16, shp, "x")
+    _check(lib.fva_inverse_reorder(_ptr(xr), _ptr(x), g.c(), _stream(stream)))
+
+
+def fva_route_workspace_size(g: Geom) -> int:
+    return int(lib.fva_route_workspace_size(g.c()))
+
+
+def fva_route(qr, kr, g: Geom, p: float, k: int, topp_mask, topk_idx, workspace, logits_out=None, stream=None):
+    shp = (g.B, g.H, g.N, g.d)
+    _need(qr, torch.bfloat16, shp, "qr")
+    _need(kr, torch.bfloat16, shp, "kr")
+    _need(topp_mask, torch.uint8, (g.B, g.H, g.Nb, g.Nb), "topp_mask")
+    _need(topk_idx, torch.int32, (g.B, g.H, g.Nb, min(k, g.Nb)), "topk_idx")
+    if logits_out is not None:
+        _need(logits_out, torch.float64, (g.B, g.H, g.Nb, g.Nb), "logits_out")
+    _check(lib.fva_route(_ptr(qr), _ptr(kr), g.c(), float(p), int(k), _ptr(topp_mask), _ptr(topk_idx),
+                         _ptr(logits_out), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                         _stream(stream)))
+
+
+def fva_repair_workspace_size(g: Geom) -> int:
+    return int(lib.fva_repair_workspace_size(g.c()))
+
+
+def fva_repair(topp_mask, topk_idx, g: Geom, k: int, counts, idx, head_work, worklist, workspace=None, stream=None):
+    _need(topp_mask, torch.uint8, (g.B, g.H, g.Nb, g.Nb), "topp_mask")
+    _need(topk_idx, torch.int32, (g.B, g.H, g.Nb, min(k, g.Nb)), "topk_idx")
+    _need(counts, torch.int32, (g.B, g.H, g.Nb), "counts")
+    _need(idx, torch.int32, (g.B, g.H, g.Nb, g.Nb), "idx")
+    _need(head_work, torch.int64, (g.B, g.H), "head_work")
+    _need(worklist, torch.int32, (g.B * g.H * g.Nb,), "worklist")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.fva_repair(_ptr(topp_mask), _ptr(topk_idx), g.c(), int(k), _ptr(counts), _ptr(idx), _ptr(head_work),
+                          _ptr(worklist), _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def fva_block_sparse_attn(qr, kr, vr, counts, idx, worklist, g: Geom, softmax_scale: float, out_r, stream=None):
+    shp = (g.B, g.H, g.N, g.d)
+    for t, n in ((qr, "qr"), (kr, "kr"), (vr, "vr"), (out_r, "out_r")):
+        _need(t, torch.bfloat16, shp, n)
+    _need(counts, torch.int32, (g.B, g.H, g.Nb), "counts")
+    _need(idx, torch.int32, (g.B, g.H, g.Nb, g.Nb), "idx")
+    if worklist is not None:
+        _need(worklist, torch.int32, (g.B * g.H * g.Nb,), "worklist")
+    _check(lib.fva_block_sparse_attn(_ptr(qr), _ptr(kr), _ptr(vr), _ptr(counts), _ptr(idx), _ptr(worklist), g.c(),
+                                     float(softmax_scale), _ptr(out_r), _stream(stream)))
+
+
+def fva_get_device_error(stream=None) -> int:
+    """Synchronises the stream; returns (and clears) the device error word, 0 if none."""
+    code = ctypes.c_int32(0)
+    rc = lib.fva_get_device_error(_stream(stream), ctypes.byref(code))
+    if rc == FVA_ERR_CUDA:
+        raise FvaError(rc, lib.fva_last_error().decode())
+    return int(code.value)
+
+
+def fva_last_error() -> str:
+    return lib.fva_last_error().decode()
+
+
+def fva_launch_count() -> int:
+    return int(lib.fva_launch_count())
+
+
+def fva_version() -> int:
+    return int(lib.fva_version())
+
+
+# ------------------------------------------------------------------ the whole path ---
+@dataclasses.dataclass
+class RouteOutputs:
+    topp_mask: torch.Tensor
+    topk_idx: torch.Tensor
+
+
+@dataclasses.dataclass
+class RepairOutputs:
+    counts: torch.Tensor
+    idx: torch.Tensor
+    head_work: torch.Tensor
+    worklist: torch.Tensor
+
+
+class SparseAttention:
+    """The whole path on one device with buffers held across calls:
+    reorder(Q, K, V) -> route -> repair -> block-sparse attention -> inverse reorder.
+
+    Buffers are allocated once through PyTorch for a geometry; `__call__` only
+    enqueues library kernels on the current (or given) stream.
+    """
+
+    def __init__(self, g: Geom, p: float, k: int, device="cuda", use_lpt: bool = True,
+                 softmax_scale: float = 0.0):
+        self.g, self.p, self.k, self.use_lpt, self.scale = g, p, k, use_lpt, softmax_scale
+        dev = torch.device(device)
+        shp = (g.B, g.H, g.N, g.d)
+        self.qr, self.kr, self.vr, self.outr = (torch.empty(shp, dtype=torch.bfloat16, device=dev) for _ in range(4))
+        kk = min(k, g.Nb)
+        self.route = RouteOutputs(torch.empty((g.B, g.H, g.Nb, g.Nb), dtype=torch.uint8, device=dev),
+                                  torch.empty((g.B, g.H, g.Nb, kk), dtype=torch.int32, device=dev))
+        self.rep = RepairOutputs(torch.empty((g.B, g.H, g.Nb), dtype=torch.int32, device=dev),
+                                 torch.empty((g.B, g.H, g.Nb, g.Nb), dtype=torch.int32, device=dev),
+                                 torch.empty((g.B, g.H), dtype=torch.int64, device=dev),
+                                 torch.empty((g.B * g.H * g.Nb,), dtype=torch.int32, device=dev))
+        self.ws = torch.empty((max(fva_route_workspace_size(g), 256),), dtype=torch.uint8, device=dev)
+
+    def routing(self, stream=None) -> None:
+        g = self.g
+        fva_route(self.qr, self.kr, g, self.p, self.k, self.route.topp_mask, self.route.topk_idx, self.ws,
+                  stream=stream)
+        fva_repair(self.route.topp_mask, self.route.topk_idx, g, self.k, self.rep.counts, self.rep.idx,
+                   self.rep.head_work, self.rep.worklist, stream=stream)
+
+    def attention(self, stream=None) -> None:
+        fva_block_sparse_attn(self.qr, self.kr, self.vr, self.rep.counts, self.rep.idx,
+                              self.rep.worklist if self.use_lpt else None, self.g, self.scale, self.outr,
+                              stream=stream)
+
+    def __call__(self, q, k, v, out, stream=None) -> torch.Tensor:
+        g = self.g
+        fva_reorder(q, self.qr, g, stream)
+        fva_reorder(k, self.kr, g, stream)
+        fva_reorder(v, self.vr, g, stream)
+        self.routing(stream)
+        self.attention(stream)
+        fva_inverse_reorder(self.outr, out, g, stream)
+        return out

@@ -1,0 +1,205 @@
+// C ABI entry points: argument validation, workspace carving and kernel launches.
+// Nothing here allocates device memory or synchronises (except fva_get_device_error).
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+
+#include <atomic>
+
+#include "fva_common.cuh"
+#include "fva_internal.h"
+
+namespace {
+
+thread_local char g_err[512] = "";
+std::atomic<long long> g_launches{0};
+
+__device__ int g_dev_err = 0;   // device error word (fva::kDevErr*)
+
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* where) {
+  return fail(FVA_ERR_CUDA, "%s: %s (%s)", where, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+int* dev_err_ptr() {
+  // per device: the symbol's address differs between devices
+  static int* ptrs[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_dev_err) != cudaSuccess) return nullptr;
+    ptrs[dev] = static_cast<int*>(p);
+  }
+  return ptrs[dev];
+}
+
+// Validates the geometry; fills D.  Returns FVA_OK or an error code (message set).
+int check_geom(const fva_geom& g, fva::Dims& D, bool need_attn_shapes) {
+  if (g.B <= 0 || g.H <= 0 || g.T <= 0 || g.Y <= 0 || g.X <= 0 || g.d <= 0 || g.tt <= 0 || g.ty <= 0 || g.tx <= 0)
+    return fail(FVA_ERR_INVALID_ARG, "geometry sizes must be positive");
+  if (g.T % g.tt || g.Y % g.ty || g.X % g.tx)
+    return fail(FVA_ERR_INVALID_ARG, "latent grid %dx%dx%d is not divisible by tile %dx%dx%d", g.T, g.Y, g.X, g.tt,
+                g.ty, g.tx);
+  const long long N = static_cast<long long>(g.T) * g.Y * g.X;
+  const long long S = static_cast<long long>(g.tt) * g.ty * g.tx;
+  const long long rows = static_cast<long long>(g.B) * g.H * N;
+  if (rows > (1LL << 31) - 1 || N > (1LL << 30))
+    return fail(FVA_ERR_INVALID_ARG, "too many tokens (B*H*N must fit in int32)");
+  if (g.d != 64 && g.d != 128) return fail(FVA_ERR_UNSUPPORTED, "head_dim %d not supported (64 or 128)", g.d);
+  if (S > 4096) return fail(FVA_ERR_UNSUPPORTED, "tile of %lld tokens not supported (<= 4096)", S);
+  if (need_attn_shapes && S != 64 && S != 128)
+    return fail(FVA_ERR_UNSUPPORTED, "tile of %lld tokens not supported (64 or 128)", S);
+  D.B = g.B;
+  D.H = g.H;
+  D.N = static_cast<int>(N);
+  D.d = g.d;
+  D.S = static_cast<int>(S);
+  D.Nb = static_cast<int>(N / S);
+  D.nT = g.T / g.tt;
+  D.nY = g.Y / g.ty;
+  D.nX = g.X / g.tx;
+  return FVA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int finish(cudaError_t e, int launches, const char* where) {
+  g_launches += launches;
+  if (e != cudaSuccess) return cuda_fail(e, where);
+  g_err[0] = '\0';
+  return FVA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t fva_version(void) { return 100; }
+
+const char* fva_last_error(void) { return g_err; }
+
+int64_t fva_launch_count(void) { return g_launches.load(); }
+
+static int reorder_common(const void* src, void* dst, fva_geom g, void* stream, bool inverse) {
+  fva::Dims D;
+  int rc = check_geom(g, D, false);
+  if (rc) return rc;
+  if (!src || !dst) return fail(FVA_ERR_INVALID_ARG, "null tensor pointer");
+  if (src == dst) return fail(FVA_ERR_INVALID_ARG, "in-place reorder is not supported");
+  if (!aligned16(src) || !aligned16(dst)) return fail(FVA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  int launches = 0;
+  cudaError_t e = fva::launch_reorder(src, dst, g, D, inverse, static_cast<cudaStream_t>(stream), &launches);
+  return finish(e, launches, inverse ? "fva_inverse_reorder" : "fva_reorder");
+}
+
+int fva_reorder(const void* x, void* xr, fva_geom g, void* stream) { return reorder_common(x, xr, g, stream, false); }
+
+int fva_inverse_reorder(const void* xr, void* x, fva_geom g, void* stream) {
+  return reorder_common(xr, x, g, stream, true);
+}
+
+size_t fva_route_workspace_size(fva_geom g) {
+  fva::Dims D;
+  if (check_geom(g, D, false)) return 0;
+  return fva::route_workspace_bytes(D);
+}
+
+int fva_route(const void* qr, const void* kr, fva_geom g, double p, int32_t k, uint8_t* topp_mask, int32_t* topk_idx,
+              double* logits_out, void* workspace, size_t workspace_bytes, void* stream) {
+  fva::Dims D;
+  int rc = check_geom(g, D, false);
+  if (rc) return rc;
+  if (!qr || !kr || !topp_mask || !topk_idx || !workspace) return fail(FVA_ERR_INVALID_ARG, "null pointer");
+  if (!(p > 0.0) || !(p <= 1.0)) return fail(FVA_ERR_INVALID_ARG, "p must satisfy 0 < p <= 1 (got %g)", p);
+  if (k < 1) return fail(FVA_ERR_INVALID_ARG, "k must be >= 1 (got %d)", k);
+  if (D.Nb > fva::kMaxNb) return fail(FVA_ERR_UNSUPPORTED, "Nb = %d blocks exceeds %d", D.Nb, fva::kMaxNb);
+  if (!aligned16(qr) || !aligned16(kr)) return fail(FVA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(FVA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  const size_t need = fva::route_workspace_bytes(D);
+  if (workspace_bytes < need)
+    return fail(FVA_ERR_INVALID_ARG, "workspace too small: %zu bytes given, %zu needed", workspace_bytes, need);
+  const int kk = k < D.Nb ? k : D.Nb;
+  int launches = 0;
+  cudaError_t e = fva::launch_route(qr, kr, D, p, kk, topp_mask, topk_idx, logits_out, workspace,
+                                    static_cast<cudaStream_t>(stream), &launches);
+  return finish(e, launches, "fva_route");
+}
+
+size_t fva_repair_workspace_size(fva_geom g) {
+  (void)g;
+  return 0;
+}
+
+int fva_repair(const uint8_t* topp_mask, const int32_t* topk_idx, fva_geom g, int32_t k, int32_t* counts, int32_t* idx,
+               int64_t* head_work, int32_t* worklist, void* workspace, size_t workspace_bytes, void* stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  fva::Dims D;
+  int rc = check_geom(g, D, false);
+  if (rc) return rc;
+  if (!topp_mask || !topk_idx || !counts || !idx || !head_work || !worklist)
+    return fail(FVA_ERR_INVALID_ARG, "null pointer");
+  if (k < 1) return fail(FVA_ERR_INVALID_ARG, "k must be >= 1 (got %d)", k);
+  if (D.Nb > fva::kMaxNb) return fail(FVA_ERR_UNSUPPORTED, "Nb = %d blocks exceeds %d", D.Nb, fva::kMaxNb);
+  int* de = dev_err_ptr();
+  if (!de) return fail(FVA_ERR_CUDA, "fva_repair: cannot resolve the device error word");
+  const int kk = k < D.Nb ? k : D.Nb;
+  int launches = 0;
+  cudaError_t e = fva::launch_repair(topp_mask, topk_idx, D, kk, counts, idx, head_work, worklist, de,
+                                     static_cast<cudaStream_t>(stream), &launches);
+  return finish(e, launches, "fva_repair");
+}
+
+int fva_block_sparse_attn(const void* qr, const void* kr, const void* vr, const int32_t* counts, const int32_t* idx,
+                          const int32_t* worklist, fva_geom g, float softmax_scale, void* out_r, void* stream) {
+  fva::Dims D;
+  int rc = check_geom(g, D, true);
+  if (rc) return rc;
+  if (!qr || !kr || !vr || !counts || !idx || !out_r) return fail(FVA_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(qr) || !aligned16(kr) || !aligned16(vr) || !aligned16(out_r))
+    return fail(FVA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  if (!isfinite(softmax_scale)) return fail(FVA_ERR_INVALID_ARG, "softmax_scale must be finite");
+  const float scale = softmax_scale > 0.0f ? softmax_scale : 1.0f / sqrtf(static_cast<float>(D.d));
+  int* de = dev_err_ptr();
+  if (!de) return fail(FVA_ERR_CUDA, "fva_block_sparse_attn: cannot resolve the device error word");
+  char msg[256] = "";
+  int launches = 0;
+  cudaError_t e = fva::launch_attention(qr, kr, vr, counts, idx, worklist, D, scale, out_r, de,
+                                        static_cast<cudaStream_t>(stream), &launches, msg, sizeof(msg));
+  if (msg[0]) {
+    g_launches += launches;
+    return fail(FVA_ERR_CUDA, "fva_block_sparse_attn: %s", msg);
+  }
+  return finish(e, launches, "fva_block_sparse_attn");
+}
+
+int fva_get_device_error(void* stream, int32_t* code) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "fva_get_device_error");
+  int* de = dev_err_ptr();
+  if (!de) return fail(FVA_ERR_CUDA, "fva_get_device_error: cannot resolve the device error word");
+  int v = 0;
+  e = cudaMemcpy(&v, de, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "fva_get_device_error");
+  if (v) {
+    const int zero = 0;
+    e = cudaMemcpy(de, &zero, sizeof(int), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_fail(e, "fva_get_device_error");
+  }
+  if (code) *code = v;
+  if (v == fva::kDevErrTimeout) return fail(FVA_ERR_TIMEOUT, "a bounded device wait expired");
+  if (v) return fail(FVA_ERR_INVALID_ARG, "a kernel rejected its input (device error %d)", v);
+  g_err[0] = '\0';
+  return FVA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,39 @@
+// Host-side launchers shared between the API translation unit and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/fva.h"
+
+namespace fva {
+
+// Derived sizes of a validated geometry.
+struct Dims {
+  int B, H, N, d, S, Nb, nT, nY, nX;
+  long long BH() const { return static_cast<long long>(B) * H; }
+  long long rows() const { return BH() * Nb; }   // (b, h, query-block) rows / work items
+};
+
+constexpr int kMaxNb = 2048;
+
+// Reorder / inverse reorder of one bf16 [B,H,N,d] tensor.
+cudaError_t launch_reorder(const void* src, void* dst, const fva_geom& g, const Dims& D, bool inverse,
+                           cudaStream_t s, int* launches);
+
+// Routing: block means (float64), float64 logits, then the Top-p / Top-k selection.
+cudaError_t launch_route(const void* qr, const void* kr, const Dims& D, double p, int kk, uint8_t* topp_mask,
+                         int32_t* topk_idx, double* logits_out, void* ws, cudaStream_t s, int* launches);
+size_t route_workspace_bytes(const Dims& D);
+
+// Repair + compaction + per-head work + LPT work list.
+cudaError_t launch_repair(const uint8_t* topp_mask, const int32_t* topk_idx, const Dims& D, int kk, int32_t* counts,
+                          int32_t* idx, int64_t* head_work, int32_t* worklist, int* dev_err, cudaStream_t s,
+                          int* launches);
+
+// Block-sparse attention (tcgen05).
+cudaError_t launch_attention(const void* qr, const void* kr, const void* vr, const int32_t* counts, const int32_t* idx,
+                             const int32_t* worklist, const Dims& D, float scale, void* out, int* dev_err,
+                             cudaStream_t s, int* launches, char* msg, size_t msg_len);
+
+}  // namespace fva

@@ -1,0 +1,146 @@
+/*
+ * fva.h — C ABI of the B200 (sm_100a) adaptive block-sparse attention path.
+ *
+ * The method is the one of "FVAttn: Adaptive Sparse Attention with Runtime Load
+ * Balancing for Video Generation" (abstract; §2 background on dynamic block-sparse
+ * routing; §3.1 pipeline overview), restricted to one GPU:
+ *
+ *   fva_reorder          video-aware block organisation: latent T x Y x X tokens -> 3D tiles
+ *   fva_route            pooled Q/K block scores, Top-p CDF cut, Top-k floor
+ *   fva_repair           forced diagonal + floor, compaction into per-row key-block lists,
+ *                        per-head realised workload, heavy-first (LPT) work list
+ *   fva_block_sparse_attn  flash-style attention over the kept block pairs
+ *   fva_inverse_reorder  back to natural token order
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - All tensor pointers are DEVICE pointers owned by the caller; nothing here
+ *   allocates device memory.  Scratch comes from a caller-provided workspace whose
+ *   size the matching *_workspace_size() query returns (bytes, 256-aligned start).
+ * - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *   Every call only enqueues work on that stream and returns; nothing synchronises
+ *   except fva_get_device_error().
+ * - bf16 tensors hold IEEE bfloat16 bit patterns.  "[B,H,N,d]" means row-major,
+ *   d fastest, N = T*Y*X tokens, contiguous, 16-byte aligned.
+ * - Token order: natural n = (t*Y + y)*X + x.  Reordered position n' = b*S + r with
+ *   b the raster index of the tile over (T/tt, Y/ty, X/tx) and r the raster index of
+ *   the token inside the tile over (tt, ty, tx); S = tt*ty*tx, Nb = N/S.
+ * - Return value: FVA_OK or an FVA_ERR_* code; on error nothing was enqueued and
+ *   fva_last_error() (thread-local) describes it.
+ */
+#ifndef FVA_H
+#define FVA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  FVA_OK = 0,
+  FVA_ERR_INVALID_ARG = 1,   /* null pointer, non-positive size, grid not divisible by tile, p/k out of range, short workspace */
+  FVA_ERR_UNSUPPORTED = 2,   /* a valid request this build does not implement (see each call) */
+  FVA_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed; fva_last_error() has the CUDA message */
+  FVA_ERR_TIMEOUT = 4        /* a bounded device-side wait expired (reported by fva_get_device_error) */
+};
+
+/* Problem geometry: batch B, heads H, latent grid T x Y x X, head_dim d, tile tt x ty x tx. */
+typedef struct fva_geom {
+  int32_t B, H, T, Y, X, d, tt, ty, tx;
+} fva_geom;
+
+/*
+ * fva_reorder — video-aware block organisation (abstract; §3.1 overview, block
+ * reordering; tiles are 3D boxes numbered in raster order).
+ *   x  : bf16 [B,H,N,d] natural order (input).
+ *   xr : bf16 [B,H,N,d] tile-major order (output): xr[.., b*S + r, :] = x[.., n(b, r), :].
+ * Exact copy.  Requires T%tt == Y%ty == X%tx == 0, d in {64, 128}, x != xr.
+ */
+int fva_reorder(const void* x, void* xr, fva_geom g, void* stream);
+
+/*
+ * fva_inverse_reorder — the inverse permutation of fva_reorder (restores natural
+ * token order on the output; §3.1 overview, final stage).  Same constraints.
+ */
+int fva_inverse_reorder(const void* xr, void* x, fva_geom g, void* stream);
+
+/* Workspace bytes fva_route needs for geometry g (pooled Q/K and block logits, float64). */
+size_t fva_route_workspace_size(fva_geom g);
+
+/*
+ * fva_route — routing frontend (§2 background: block importance and binary mask;
+ * Top-p retains the fewest key blocks whose summed normalised importance is >= p;
+ * Top-k floor; §3.1 overview: block similarities from pooled Q/K).
+ *   qr, kr     : bf16 [B,H,N,d], tile-major (fva_reorder output).
+ *   p          : Top-p threshold, 0 < p <= 1 (p >= 1 keeps every block).
+ *   k          : Top-k floor, k >= 1 (clamped to Nb).
+ *   topp_mask  : uint8 [B,H,Nb,Nb] output, 1 where key block j is in row i's Top-p set.
+ *   topk_idx   : int32 [B,H,Nb,min(k,Nb)] output, the min(k,Nb) highest-ranked key
+ *                blocks of each row, in ascending block id.
+ *   logits_out : optional float64 [B,H,Nb,Nb] output of Qbar_i.Kbar_j/sqrt(d), or NULL.
+ * Arithmetic: per-block means and logits in float64; rows ranked by logit descending,
+ * ties to the lower block id; the cumulative mass of the softmax is accumulated in
+ * 2^-62 fixed point, so the result is deterministic.  Requires Nb <= 2048.
+ */
+int fva_route(const void* qr, const void* kr, fva_geom g, double p, int32_t k,
+              uint8_t* topp_mask, int32_t* topk_idx, double* logits_out,
+              void* workspace, size_t workspace_bytes, void* stream);
+
+/* Workspace bytes fva_repair needs (currently 0; kept for ABI stability). */
+size_t fva_repair_workspace_size(fva_geom g);
+
+/*
+ * fva_repair — runtime mask repair and compaction (abstract: the materialised mask
+ * is repaired at run time; §2 sequence parallelism: realised per-head workload).
+ *   topp_mask, topk_idx, k : fva_route outputs and the same k.
+ *   counts    : int32 [B,H,Nb] output, kept key blocks per query block (>= 1).
+ *   idx       : int32 [B,H,Nb,Nb] output; row (b,h,i) holds counts[b,h,i] ascending key
+ *               block ids in its first entries; entries past the count are not written.
+ *   head_work : int64 [B,H] output, W_h = sum over i of counts (kept block pairs).
+ *   worklist  : int32 [B*H*Nb] output, item ids u = (b*H + h)*Nb + i ordered by count
+ *               descending, ties by u ascending (longest processing time first).
+ * Kept set of row i = Top-p set U Top-k floor U {i}.  Requires Nb <= 2048.
+ */
+int fva_repair(const uint8_t* topp_mask, const int32_t* topk_idx, fva_geom g, int32_t k,
+               int32_t* counts, int32_t* idx, int64_t* head_work, int32_t* worklist,
+               void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * fva_block_sparse_attn — block-sparse flash attention over the kept pairs (§3.1
+ * overview: block-sparse attention after routing; §2: only selected block pairs
+ * are evaluated).  Bidirectional, no causal mask.
+ *   qr, kr, vr : bf16 [B,H,N,d] tile-major.
+ *   counts,idx : fva_repair outputs (every listed id must be in [0, Nb)).
+ *   worklist   : fva_repair's LPT order, or NULL for item-id order.
+ *   softmax_scale : <= 0 selects 1/sqrt(d).
+ *   out_r      : bf16 [B,H,N,d] tile-major output, O_i = softmax(Q_i K_J^T * scale) V_J
+ *                over the union J of the kept key blocks of query block i.
+ * tcgen05 tensor-core MMAs (bf16 in, fp32 accumulate in TMEM), fp32 online softmax,
+ * bf16 round-to-nearest output.  Requires d in {64, 128} and S = tt*ty*tx in {64, 128}.
+ */
+int fva_block_sparse_attn(const void* qr, const void* kr, const void* vr,
+                          const int32_t* counts, const int32_t* idx, const int32_t* worklist,
+                          fva_geom g, float softmax_scale, void* out_r, void* stream);
+
+/*
+ * fva_get_device_error — synchronises `stream`, then reads and clears the device
+ * error word that bounded waits inside the kernels set.  *code receives the raw
+ * word (0 = none).  Returns FVA_OK, FVA_ERR_TIMEOUT if a wait expired, or FVA_ERR_CUDA.
+ */
+int fva_get_device_error(void* stream, int32_t* code);
+
+/* Thread-local description of the last error returned on this thread ("" if none). */
+const char* fva_last_error(void);
+
+/* Number of kernel launches this library has enqueued since load (process-wide). */
+int64_t fva_launch_count(void);
+
+/* ABI version (major*100 + minor). */
+int32_t fva_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FVA_H */

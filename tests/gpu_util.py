@@ -1,0 +1,91 @@
+"""Helpers for the GPU parity tests: move seeded bf16 inputs to the device, run the
+library path step by step, and compare with the oracle under the parity rules
+(bit-exact integer work modulo flagged ties; attention within max-abs 2e-2 and
+relative-L2 5e-3 with the device's own index lists fed to the oracle)."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle as O
+
+ATOL = 2e-2
+REL_L2 = 5e-3
+
+
+def to_dev(bits: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def to_bits(t: torch.Tensor) -> np.ndarray:
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def bf16_dev_to_f64(t: torch.Tensor) -> np.ndarray:
+    return O.bf16_bits_to_f64(to_bits(t))
+
+
+def run_path(fva, g, q, k, v, p, kfloor, use_lpt=True, want_logits=False):
+    """Runs every library step; returns a dict of device results (torch tensors)."""
+    dev = {}
+    qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
+    shp = (g.B, g.H, g.N, g.d)
+    qr, kr, vr, outr, out = (torch.empty(shp, dtype=torch.bfloat16, device="cuda") for _ in range(5))
+    fva.fva_reorder(qd, qr, g)
+    fva.fva_reorder(kd, kr, g)
+    fva.fva_reorder(vd, vr, g)
+    kk = min(kfloor, g.Nb)
+    mask = torch.empty((g.B, g.H, g.Nb, g.Nb), dtype=torch.uint8, device="cuda")
+    topk = torch.empty((g.B, g.H, g.Nb, kk), dtype=torch.int32, device="cuda")
+    ws = torch.empty((fva.fva_route_workspace_size(g),), dtype=torch.uint8, device="cuda")
+    logits = torch.empty((g.B, g.H, g.Nb, g.Nb), dtype=torch.float64, device="cuda") if want_logits else None
+    fva.fva_route(qr, kr, g, p, kfloor, mask, topk, ws, logits_out=logits)
+    counts = torch.empty((g.B, g.H, g.Nb), dtype=torch.int32, device="cuda")
+    idx = torch.full((g.B, g.H, g.Nb, g.Nb), -1, dtype=torch.int32, device="cuda")
+    hw = torch.empty((g.B, g.H), dtype=torch.int64, device="cuda")
+    wl = torch.empty((g.B * g.H * g.Nb,), dtype=torch.int32, device="cuda")
+    fva.fva_repair(mask, topk, g, kfloor, counts, idx, hw, wl)
+    fva.fva_block_sparse_attn(qr, kr, vr, counts, idx, wl if use_lpt else None, g, 0.0, outr)
+    fva.fva_inverse_reorder(outr, out, g)
+    torch.cuda.synchronize()
+    assert fva.fva_get_device_error() == 0
+    dev.update(qr=qr, kr=kr, vr=vr, mask=mask, topk=topk, logits=logits, counts=counts, idx=idx, head_work=hw,
+               worklist=wl, outr=outr, out=out)
+    return dev
+
+
+def check_route(rr: O.RouteResult, mask_dev: np.ndarray, topk_dev: np.ndarray, max_tie_frac=0.02):
+    """Bit-exact comparison except rows flagged as ties; returns (n_rows, n_tie_rows, n_diff_rows)."""
+    t1, t2p, t2k = O.tie_flags(rr)
+    dm = (mask_dev != rr.topp_mask).any(-1)
+    dk = (topk_dev != rr.topk_idx).any(-1)
+    bad_m = dm & ~(t1 | t2p)
+    bad_k = dk & ~t2k
+    assert not bad_m.any(), f"{int(bad_m.sum())} Top-p rows differ without a tie, e.g. {np.argwhere(bad_m)[:5]}"
+    assert not bad_k.any(), f"{int(bad_k.sum())} Top-k rows differ without a tie, e.g. {np.argwhere(bad_k)[:5]}"
+    ties = t1 | t2p | t2k
+    assert ties.mean() <= max_tie_frac, f"tie rows {ties.mean():.4f} above {max_tie_frac}"
+    return int(ties.size), int(ties.sum()), int((dm | dk).sum())
+
+
+def check_repair(fva_dev: dict, mask_dev: np.ndarray, topk_dev: np.ndarray):
+    """The device repair outputs equal the oracle repair of the device's own route outputs, exactly."""
+    rp = O.repair(mask_dev, topk_dev)
+    counts = fva_dev["counts"].cpu().numpy()
+    idx = fva_dev["idx"].cpu().numpy()
+    assert np.array_equal(counts, rp.counts)
+    B, H, Nb = counts.shape
+    valid = np.arange(Nb)[None, None, None, :] < counts[..., None]
+    assert np.array_equal(np.where(valid, idx, -1), rp.idx)
+    assert np.array_equal(fva_dev["head_work"].cpu().numpy(), rp.head_work)
+    assert np.array_equal(fva_dev["worklist"].cpu().numpy(), rp.worklist)
+    return rp
+
+
+def compare_attention(got: np.ndarray, want: np.ndarray):
+    err = np.abs(got - want)
+    mx = float(err.max()) if err.size else 0.0
+    rel = float(np.linalg.norm(got - want) / max(np.linalg.norm(want), 1e-30))
+    assert mx <= ATOL, f"max-abs {mx:.3e} > {ATOL}"
+    assert rel <= REL_L2, f"rel-L2 {rel:.3e} > {REL_L2}"
+    return mx, rel

@@ -1,0 +1,97 @@
+"""Host-side checks of the C ABI: the library loads, exports every entry point the
+header declares, and rejects bad arguments before touching the GPU.  CPU only."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import block_sparse_attention_44_b200 as fva
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if f.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", f)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(fva_[a-z0-9_]+)\s*\(", src))
+    return names
+
+
+def test_every_declared_symbol_is_exported():
+    names = _declared()
+    assert {"fva_reorder", "fva_inverse_reorder", "fva_route", "fva_repair", "fva_block_sparse_attn"} <= names
+    raw = ctypes.CDLL(fva.LIB_PATH)
+    for n in sorted(names):
+        assert hasattr(raw, n), n
+
+
+def test_version_and_counters():
+    assert fva.fva_version() >= 100
+    assert fva.fva_launch_count() >= 0
+
+
+def _g(**kw):
+    base = dict(B=1, H=2, T=4, Y=8, X=8, d=64, tt=1, ty=8, tx=8)
+    base.update(kw)
+    return fva.Geom(**base)
+
+
+def test_workspace_size_queries():
+    g = _g()
+    # pooled Q and K (float64) plus the float64 logits, each 256-byte aligned
+    nb = g.Nb
+    rows = g.B * g.H * nb
+    def al(x):
+        return (x + 255) // 256 * 256
+    assert fva.fva_route_workspace_size(g) == 2 * al(rows * g.d * 8) + al(rows * nb * 8)
+    assert fva.fva_repair_workspace_size(g) == 0
+    assert fva.fva_route_workspace_size(_g(X=9)) == 0          # invalid geometry
+
+
+def _rc(fn, *args):
+    return fn(*args)
+
+
+def test_invalid_arguments_rejected_on_host():
+    L = fva.lib
+    g = _g().c()
+    assert L.fva_reorder(None, None, g, None) == fva.FVA_ERR_INVALID_ARG
+    assert b"null" in L.fva_last_error()
+    bad = _g(X=9).c()
+    assert L.fva_reorder(16, 32, bad, None) == fva.FVA_ERR_INVALID_ARG
+    assert b"divisible" in L.fva_last_error()
+    assert L.fva_reorder(16, 16, g, None) == fva.FVA_ERR_INVALID_ARG           # in place
+    assert L.fva_reorder(17, 32, g, None) == fva.FVA_ERR_INVALID_ARG           # misaligned
+    assert L.fva_reorder(16, 32, _g(d=96).c(), None) == fva.FVA_ERR_UNSUPPORTED
+    assert L.fva_reorder(16, 32, _g(B=0).c(), None) == fva.FVA_ERR_INVALID_ARG
+    # route: p and k ranges, workspace size and alignment
+    args = lambda p, k, ws, wsb: (256, 512, g, p, k, 768, 1024, None, ws, wsb, None)
+    need = fva.fva_route_workspace_size(_g())
+    assert L.fva_route(*args(0.0, 1, 4096, need)) == fva.FVA_ERR_INVALID_ARG
+    assert L.fva_route(*args(1.5, 1, 4096, need)) == fva.FVA_ERR_INVALID_ARG
+    assert L.fva_route(*args(float("nan"), 1, 4096, need)) == fva.FVA_ERR_INVALID_ARG
+    assert L.fva_route(*args(0.9, 0, 4096, need)) == fva.FVA_ERR_INVALID_ARG
+    assert L.fva_route(*args(0.9, 1, 4096, need - 1)) == fva.FVA_ERR_INVALID_ARG
+    assert b"workspace too small" in L.fva_last_error()
+    assert L.fva_route(*args(0.9, 1, 4100, need)) == fva.FVA_ERR_INVALID_ARG  # not 256-aligned
+    # repair / attention: null pointers, k, unsupported tile for attention
+    assert L.fva_repair(None, 16, g, 1, 16, 16, 16, 16, None, 0, None) == fva.FVA_ERR_INVALID_ARG
+    assert L.fva_repair(16, 16, g, 0, 16, 16, 16, 16, None, 0, None) == fva.FVA_ERR_INVALID_ARG
+    assert L.fva_block_sparse_attn(16, 16, None, 16, 16, None, g, 0.0, 16, None) == fva.FVA_ERR_INVALID_ARG
+    t32 = _g(tt=1, ty=4, tx=8).c()                                            # 32-token tiles
+    assert L.fva_block_sparse_attn(16, 16, 16, 16, 16, None, t32, 0.0, 16, None) == fva.FVA_ERR_UNSUPPORTED
+    assert L.fva_block_sparse_attn(16, 16, 16, 16, 16, None, g, float("inf"), 16, None) == fva.FVA_ERR_INVALID_ARG
+    big = _g(T=64, Y=128, X=128, tt=1, ty=8, tx=8).c()                       # Nb = 16384 > 2048
+    assert L.fva_route(256, 512, big, 0.9, 1, 768, 1024, None, 4096, 1 << 40, None) == fva.FVA_ERR_UNSUPPORTED
+
+
+def test_python_wrapper_type_checks():
+    import torch
+    g = _g()
+    x = torch.zeros((1, 2, 256, 64), dtype=torch.float32)
+    with pytest.raises(TypeError):
+        fva.fva_reorder(x, x, g)

@@ -1,0 +1,57 @@
+"""Full-size parity: the Wan-like 480p and 720p single-layer workloads in the
+launch configuration the benchmark times (LPT work list).  Routing and repair are
+checked in full; attention on a sample of items the oracle computes one by one
+(the heaviest, the lightest and a seeded random set)."""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+import oracle as O
+import synth
+from gpu_util import bf16_dev_to_f64, check_repair, check_route, compare_attention, run_path, to_bits
+
+
+@pytest.fixture(scope="module")
+def fva():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import block_sparse_attention_44_b200 as m
+    return m
+
+
+@pytest.mark.parametrize("name", ["wan480p", "wan720p"])
+def test_fullsize(fva, name):
+    cfg = synth.CONFIGS[name]
+    g = fva.Geom.of(cfg)
+    og = O.Geometry.of(cfg)
+    q, k, v = synth.make_qkv(cfg)
+    dev = run_path(fva, g, q, k, v, cfg.p, cfg.k, use_lpt=True)
+    qr = O.reorder(q, og)
+    kr = O.reorder(k, og)
+    del q, k
+    assert np.array_equal(to_bits(dev["qr"]), qr)
+    assert np.array_equal(to_bits(dev["kr"]), kr)
+    rr = O.route(qr, kr, og, cfg.p, cfg.k)
+    mask_dev = dev["mask"].cpu().numpy()
+    topk_dev = dev["topk"].cpu().numpy()
+    n_rows, n_ties, n_diff = check_route(rr, mask_dev, topk_dev)
+    print(f"{name}: {n_rows} rows, {n_ties} tie-flagged, {n_diff} differing (all flagged)")
+    rp = check_repair(dev, mask_dev, topk_dev)
+    density = rp.counts.sum() / (og.B * og.H * og.Nb * og.Nb)
+    print(f"{name}: density {density:.4f}")
+    vr = O.reorder(v, og)
+    wl = rp.worklist
+    rng = np.random.default_rng(0)
+    pick = np.concatenate([wl[:8], wl[-8:], rng.choice(wl, size=16, replace=False)])
+    items = []
+    for u in pick.tolist():
+        b, rem = divmod(u, og.H * og.Nb)
+        h, i = divmod(rem, og.Nb)
+        items.append((b, h, i))
+    want = O.attention_items(qr, kr, vr, rp.counts, rp.idx, og.S, items)
+    out = dev["outr"]
+    for (b, h, i), o in want.items():
+        got = bf16_dev_to_f64(out[b, h, i * og.S:(i + 1) * og.S])
+        compare_attention(got, o)

@@ -1,0 +1,175 @@
+"""GPU path vs the CPU oracle, through the C ABI, on seeded synthetic inputs.
+
+Parity rules: reorder / inverse reorder and the repaired lists bit-exact; Top-p
+masks and Top-k lists bit-exact except rows the oracle flags as ties; attention
+with the device's own index lists fed to the oracle within max-abs 2e-2 and
+relative-L2 5e-3 of the float64 result.
+"""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+import oracle as O
+import synth
+from gpu_util import (bf16_dev_to_f64, check_repair, check_route, compare_attention, run_path, to_bits, to_dev)
+
+
+@pytest.fixture(scope="module")
+def fva():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import block_sparse_attention_44_b200 as m
+    return m
+
+
+def _cfg(name, **kw):
+    base = dict(B=1, H=2, d=128, T=4, Y=16, X=16, tt=2, ty=8, tx=8, p=0.9, k=4, a_mode="loguniform",
+                a_lo=0.5, a_hi=4.0, noise_std=1.0, sigma=0.3, seed=0)
+    base.update(kw)
+    return synth.Config(name, **base)
+
+
+CASES = {
+    "tiny": synth.CONFIGS["tiny"],
+    # 2 x 6 x 24 = 288 items: more than one persistent wave, a ragged tail
+    "d128_s128_multiwave": _cfg("d128_s128_multiwave", B=2, H=6, T=4, Y=16, X=48, seed=1),
+    "d128_s64": _cfg("d128_s64", H=4, T=2, Y=16, X=32, tt=1, ty=8, tx=8, seed=2),
+    "d64_s128": _cfg("d64_s128", H=3, d=64, T=4, Y=16, X=16, seed=3),
+    "stress_small": _cfg("stress_small", H=4, T=4, Y=16, X=32, p=0.95, a_mode="alternating", a_lo=4.0, a_hi=0.3,
+                         seed=4),
+    "dense_p1": _cfg("dense_p1", H=3, T=4, Y=16, X=32, p=1.0, seed=5),
+    "topk_only": _cfg("topk_only", H=3, T=4, Y=16, X=32, p=1e-9, k=3, seed=6),
+    "k_above_nb": _cfg("k_above_nb", H=2, T=4, Y=16, X=16, k=50, seed=7),
+    "single_block": _cfg("single_block", H=2, T=2, Y=8, X=8, seed=8),
+}
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_path_matches_oracle(fva, name):
+    cfg = CASES[name]
+    g = fva.Geom.of(cfg)
+    og = O.Geometry.of(cfg)
+    q, k, v = synth.make_qkv(cfg)
+    dev = run_path(fva, g, q, k, v, cfg.p, cfg.k, want_logits=True)
+
+    # a1: reorder, bit-exact
+    qr, kr, vr = (O.reorder(t, og) for t in (q, k, v))
+    assert np.array_equal(to_bits(dev["qr"]), qr)
+    assert np.array_equal(to_bits(dev["kr"]), kr)
+    assert np.array_equal(to_bits(dev["vr"]), vr)
+
+    # a2-a4: routing, bit-exact modulo ties; logits to float64 rounding
+    rr = O.route(qr, kr, og, cfg.p, cfg.k)
+    L = dev["logits"].cpu().numpy()
+    assert np.allclose(L, rr.L, rtol=1e-12, atol=1e-12)
+    mask_dev = dev["mask"].cpu().numpy()
+    topk_dev = dev["topk"].cpu().numpy()
+    check_route(rr, mask_dev, topk_dev)
+    if cfg.p >= 1.0:
+        assert (mask_dev == 1).all()
+
+    # a5: repair, exact given the device's own route outputs
+    rp = check_repair(dev, mask_dev, topk_dev)
+    assert (rp.counts >= min(cfg.k, og.Nb)).all()
+
+    # a6: attention with the device index lists, all items
+    want = O.attention(qr, kr, vr, rp.counts, rp.idx, og.S)
+    got = bf16_dev_to_f64(dev["outr"])
+    compare_attention(got, want)
+
+    # a7: inverse reorder, bit-exact against the oracle's inverse of the device output
+    assert np.array_equal(to_bits(dev["out"]), O.inverse_reorder(to_bits(dev["outr"]), og))
+
+
+def test_lpt_and_static_order_identical(fva):
+    cfg = CASES["d128_s128_multiwave"]
+    g = fva.Geom.of(cfg)
+    q, k, v = synth.make_qkv(cfg)
+    a = run_path(fva, g, q, k, v, cfg.p, cfg.k, use_lpt=True)
+    b = run_path(fva, g, q, k, v, cfg.p, cfg.k, use_lpt=False)
+    assert torch.equal(a["outr"].view(torch.int16), b["outr"].view(torch.int16))
+    # repeated runs are bit-identical (deterministic routing and attention)
+    c = run_path(fva, g, q, k, v, cfg.p, cfg.k, use_lpt=True)
+    for key in ("mask", "topk", "counts", "worklist", "outr"):
+        x, y = a[key], c[key]
+        if x.dtype == torch.bfloat16:
+            x, y = x.view(torch.int16), y.view(torch.int16)
+        assert torch.equal(x, y), key
+
+
+def test_worklist_is_lpt_order(fva):
+    cfg = CASES["stress_small"]
+    g = fva.Geom.of(cfg)
+    q, k, v = synth.make_qkv(cfg)
+    dev = run_path(fva, g, q, k, v, cfg.p, cfg.k)
+    c = dev["counts"].cpu().numpy().reshape(-1)
+    wl = dev["worklist"].cpu().numpy()
+    assert sorted(wl.tolist()) == list(range(c.size))
+    assert (np.diff(c[wl]) <= 0).all()
+    assert np.array_equal(wl, O.lpt_worklist(c))
+
+
+def test_attention_handcrafted_lists(fva):
+    """Lists not produced by routing: empty rows give zeros, arbitrary order of ids, all blocks."""
+    cfg = CASES["d128_s128_multiwave"].with_(B=1, H=2)
+    g = fva.Geom.of(cfg)
+    og = O.Geometry.of(cfg)
+    q, k, v = synth.make_qkv(cfg)
+    qr, kr, vr = (O.reorder(t, og) for t in (q, k, v))
+    rng = np.random.default_rng(0)
+    Nb = og.Nb
+    counts = rng.integers(0, Nb + 1, size=(1, 2, Nb)).astype(np.int32)
+    counts[0, 0, 0] = 0
+    counts[0, 1, 3] = Nb
+    idx = np.full((1, 2, Nb, Nb), -1, dtype=np.int32)
+    for h in range(2):
+        for i in range(Nb):
+            idx[0, h, i, :counts[0, h, i]] = rng.permutation(Nb)[:counts[0, h, i]]
+    out = torch.empty((1, 2, og.N, og.d), dtype=torch.bfloat16, device="cuda")
+    fva.fva_block_sparse_attn(to_dev(qr), to_dev(kr), to_dev(vr), torch.from_numpy(counts).cuda(),
+                              torch.from_numpy(idx).cuda(), None, g, 0.0, out)
+    torch.cuda.synchronize()
+    assert fva.fva_get_device_error() == 0
+    got = bf16_dev_to_f64(out)
+    nz = counts > 0
+    items = [(0, h, i) for h in range(2) for i in range(Nb) if nz[0, h, i]]
+    want = O.attention_items(qr, kr, vr, counts, idx, og.S, items)
+    for (b, h, i), o in want.items():
+        compare_attention(got[b, h, i * og.S:(i + 1) * og.S], o)
+    for h in range(2):
+        for i in range(Nb):
+            if not nz[0, h, i]:
+                assert (got[0, h, i * og.S:(i + 1) * og.S] == 0).all()
+
+
+def test_attention_custom_scale(fva):
+    cfg = CASES["tiny"]
+    g = fva.Geom.of(cfg)
+    og = O.Geometry.of(cfg)
+    q, k, v = synth.make_qkv(cfg)
+    qr, kr, vr = (O.reorder(t, og) for t in (q, k, v))
+    Nb = og.Nb
+    counts = np.full((1, 2, Nb), Nb, dtype=np.int32)
+    idx = np.broadcast_to(np.arange(Nb, dtype=np.int32), (1, 2, Nb, Nb)).copy()
+    out = torch.empty((1, 2, og.N, og.d), dtype=torch.bfloat16, device="cuda")
+    fva.fva_block_sparse_attn(to_dev(qr), to_dev(kr), to_dev(vr), torch.from_numpy(counts).cuda(),
+                              torch.from_numpy(idx).cuda(), None, g, 0.05, out)
+    torch.cuda.synchronize()
+    compare_attention(bf16_dev_to_f64(out), O.attention(qr, kr, vr, counts, idx, og.S, scale=0.05))
+
+
+def test_out_of_range_block_id_is_reported(fva):
+    cfg = CASES["tiny"]
+    g = fva.Geom.of(cfg)
+    og = O.Geometry.of(cfg)
+    q, k, v = synth.make_qkv(cfg)
+    Nb = og.Nb
+    counts = torch.full((1, 2, Nb), 2, dtype=torch.int32, device="cuda")
+    idx = torch.zeros((1, 2, Nb, Nb), dtype=torch.int32, device="cuda")
+    idx[0, 0, 1, 1] = Nb + 5                       # out of range: the kernel substitutes the diagonal
+    out = torch.empty((1, 2, og.N, og.d), dtype=torch.bfloat16, device="cuda")
+    fva.fva_block_sparse_attn(to_dev(q), to_dev(k), to_dev(v), counts, idx, None, g, 0.0, out)
+    assert fva.fva_get_device_error() == 2
+    assert fva.fva_get_device_error() == 0         # cleared by the read
