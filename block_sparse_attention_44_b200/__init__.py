@@ -16,7 +16,7 @@ import torch
 
 __all__ = [
     "FvaError", "Geom", "lib", "fva_reorder", "fva_inverse_reorder", "fva_route_workspace_size", "fva_route",
-    "fva_repair_workspace_size", "fva_repair", "fva_block_sparse_attn", "fva_get_device_error", "fva_last_error",
+    "fva_route_static", "fva_repair_workspace_size", "fva_repair", "fva_block_sparse_attn", "fva_get_device_error", "fva_last_error",
     "fva_launch_count", "fva_version", "RouteOutputs", "RepairOutputs", "SparseAttention",
 ]
 
@@ -82,6 +82,7 @@ def _load():
         "fva_inverse_reorder": ([vp, vp, _Geom, vp], ctypes.c_int),
         "fva_route_workspace_size": ([_Geom], sz),
         "fva_route": ([vp, vp, _Geom, f64, i32, vp, vp, vp, vp, sz, vp], ctypes.c_int),
+        "fva_route_static": ([vp, vp, _Geom, f64, i32, vp, vp, vp, vp], ctypes.c_int),
         "fva_repair_workspace_size": ([_Geom], sz),
         "fva_repair": ([vp, vp, _Geom, i32, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
         "fva_block_sparse_attn": ([vp, vp, vp, vp, vp, vp, _Geom, f32, vp, vp], ctypes.c_int),
@@ -160,6 +161,26 @@ def fva_route(qr, kr, g: Geom, p: float, k: int, topp_mask, topk_idx, workspace,
     _check(lib.fva_route(_ptr(qr), _ptr(kr), g.c(), float(p), int(k), _ptr(topp_mask), _ptr(topk_idx),
                          _ptr(logits_out), _ptr(workspace), workspace.numel() * workspace.element_size(),
                          _stream(stream)))
+
+
+ROUTE_STATIC_SCRATCH_BYTES = 64 << 20
+
+
+def fva_route_static(qr, kr, g: Geom, p: float, k: int, topp_mask, topk_idx, logits_out=None, stream=None):
+    """fva_route without a workspace, for callers that cannot allocate device memory
+    (e.g. a plugin whose host framework owns all device allocations, or a serving loop
+    with a fixed memory plan).  The routing scratch is a 64 MiB device array inside the
+    library, shared by every call on a device: calls that overlap on the GPU race.
+    Larger geometries raise FvaError(FVA_ERR_UNSUPPORTED)."""
+    shp = (g.B, g.H, g.N, g.d)
+    _need(qr, torch.bfloat16, shp, "qr")
+    _need(kr, torch.bfloat16, shp, "kr")
+    _need(topp_mask, torch.uint8, (g.B, g.H, g.Nb, g.Nb), "topp_mask")
+    _need(topk_idx, torch.int32, (g.B, g.H, g.Nb, min(k, g.Nb)), "topk_idx")
+    if logits_out is not None:
+        _need(logits_out, torch.float64, (g.B, g.H, g.Nb, g.Nb), "logits_out")
+    _check(lib.fva_route_static(_ptr(qr), _ptr(kr), g.c(), float(p), int(k), _ptr(topp_mask), _ptr(topk_idx),
+                                _ptr(logits_out), _stream(stream)))
 
 
 def fva_repair_workspace_size(g: Geom) -> int:

@@ -203,3 +203,61 @@ int fva_get_device_error(void* stream, int32_t* code) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------------
+// fva_route_static: fva_route without a caller-provided workspace.
+//
+// Some callers cannot allocate device memory at the point where they route: a plugin
+// running inside a host framework that owns every device allocation and hands its
+// plugins no allocator, or a latency-critical serving loop whose memory plan is fixed
+// before it starts and where a cudaMalloc (which may synchronise the device or fail
+// under fragmentation) is not acceptable.  For them the routing scratch lives in one
+// file-scope device array of fixed size, reserved on every GPU that loads this
+// library and held until the process exits.
+// ---------------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kRouteStaticScratchBytes = FVA_ROUTE_STATIC_SCRATCH_BYTES;
+static __device__ __align__(256) unsigned char g_route_scratch[kRouteStaticScratchBytes];
+
+// Device address of g_route_scratch on the current device.  In host code the symbol
+// only names a host-side stand-in, so the address must come from the runtime; it is
+// looked up once per device, with that device current, on the first call there.
+void* route_scratch_ptr() {
+  static std::atomic<void*> ptrs[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  void* p = ptrs[dev].load();
+  if (!p) {
+    if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess) return nullptr;
+    ptrs[dev].store(p);
+  }
+  return p;
+}
+
+}  // namespace
+
+extern "C" int fva_route_static(const void* qr, const void* kr, fva_geom g, double p, int32_t k,
+                                uint8_t* topp_mask, int32_t* topk_idx, double* logits_out, void* stream) {
+  fva::Dims D;
+  int rc = check_geom(g, D, false);
+  if (rc) return rc;
+  if (!qr || !kr || !topp_mask || !topk_idx) return fail(FVA_ERR_INVALID_ARG, "null pointer");
+  if (!(p > 0.0) || !(p <= 1.0)) return fail(FVA_ERR_INVALID_ARG, "p must satisfy 0 < p <= 1 (got %g)", p);
+  if (k < 1) return fail(FVA_ERR_INVALID_ARG, "k must be >= 1 (got %d)", k);
+  if (D.Nb > fva::kMaxNb) return fail(FVA_ERR_UNSUPPORTED, "Nb = %d blocks exceeds %d", D.Nb, fva::kMaxNb);
+  if (!aligned16(qr) || !aligned16(kr)) return fail(FVA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  const size_t need = fva::route_workspace_bytes(D);
+  if (need > kRouteStaticScratchBytes)
+    return fail(FVA_ERR_UNSUPPORTED,
+                "fva_route_static: this geometry needs %zu bytes of routing scratch, more than the %zu-byte "
+                "static scratch; use fva_route with a caller workspace",
+                need, kRouteStaticScratchBytes);
+  void* scratch = route_scratch_ptr();
+  if (!scratch) return fail(FVA_ERR_CUDA, "fva_route_static: cannot resolve the static scratch address");
+  const int kk = k < D.Nb ? k : D.Nb;
+  int launches = 0;
+  cudaError_t e = fva::launch_route(qr, kr, D, p, kk, topp_mask, topk_idx, logits_out, scratch,
+                                    static_cast<cudaStream_t>(stream), &launches);
+  return finish(e, launches, "fva_route_static");
+}

@@ -88,6 +88,33 @@ int fva_route(const void* qr, const void* kr, fva_geom g, double p, int32_t k,
               uint8_t* topp_mask, int32_t* topk_idx, double* logits_out,
               void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * fva_route_static — fva_route for callers that cannot allocate device memory.
+ * The paper has no counterpart: this is a deployment variant of fva_route.
+ *
+ * Who needs it: code that routes where it may not call cudaMalloc — e.g. a plugin
+ * inside a host framework that owns every device allocation and gives plugins no
+ * allocator, or a serving loop whose device memory plan is fixed up front, where an
+ * allocation (which can synchronise the device or fail under fragmentation) is not
+ * acceptable.  Same arguments, results and arithmetic as fva_route, minus the
+ * workspace: the routing scratch is one file-scope device array of
+ * FVA_ROUTE_STATIC_SCRATCH_BYTES (64 MiB), reserved on every GPU that loads this
+ * library and held until the process exits.
+ *   - Geometries whose fva_route_workspace_size() exceeds that size are rejected with
+ *     FVA_ERR_UNSUPPORTED and a message; nothing is enqueued.  (The 480p layer,
+ *     B=1 H=40 d=128 with 240 blocks, needs about 36 MiB; the 720p layer does not fit.)
+ *   - Nothing in the scratch needs to start at zero: each call writes every scratch
+ *     byte it later reads.  The array keeps the last call's contents.
+ *   - All calls on a device share the one array: calls whose GPU execution overlaps
+ *     (different streams, no ordering between them) race and give wrong results.
+ *   - The first call on a device looks up the array's device address with that device
+ *     current (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - Allocates nothing (no cudaMalloc, cudaFree or allocating library routine).
+ */
+#define FVA_ROUTE_STATIC_SCRATCH_BYTES ((size_t)64 << 20)
+int fva_route_static(const void* qr, const void* kr, fva_geom g, double p, int32_t k,
+                     uint8_t* topp_mask, int32_t* topk_idx, double* logits_out, void* stream);
+
 /* Workspace bytes fva_repair needs (currently 0; kept for ABI stability). */
 size_t fva_repair_workspace_size(fva_geom g);
 
