@@ -5,16 +5,22 @@
 //
 // Persistent kernel, one CTA per SM, walking a work list of (b, h, query-block)
 // items (heavy items first when the caller passes the LPT list).  Per item the CTA
-// keeps the 128-row Q tile in shared memory and streams the item's kept K/V blocks
-// through an NS-stage TMA ring.  Roles (8 warps):
-//   warp 0  : TMA producer (one thread)        — Q once per item, K_j and V_j per block
-//   warp 1  : MMA issuer (one thread)          — S_j = Q K_j^T (SS), O += P_j V_j (TS)
-//   warp 2  : TMEM allocator
-//   warps 4-7: softmax / correction / epilogue — thread r owns query row r (TMEM lane r)
-// Tensor memory: two S buffers (double-buffered so S_{j+1} overlaps softmax j; the
-// bf16 P_j overwrites the first half of its own S buffer and feeds the TS MMA) and
-// the fp32 O accumulator.  Online softmax in base 2 with a lazy running max: O and
-// the row sum are rescaled only when the max grows by more than 2^8.
+// keeps the 128-row Q tile in shared memory and streams the item's kept K and V
+// blocks through two TMA rings; a K stage is released as soon as its S product is
+// done, a V stage after its PV product.  Roles (12 warps):
+//   warp 0    : TMA producer  — Q once per item, K_j per kept block
+//   warp 3    : TMA producer  — V_j per kept block
+//   warp 1    : MMA issuer    — S_j = Q K_j^T (both operands in shared memory)
+//   warp 2    : MMA issuer    — O += P_j V_j (P from tensor memory); allocates TMEM
+//   warps 4-11: softmax, O correction and epilogue — two warps per TMEM lane
+//               quarter, each owning half of the columns of its 32 query rows
+// One thread can issue a tcgen05.mma only about as fast as a 128x128x16 product
+// runs, so the two kinds of product come from two warps on different SM
+// sub-partitions and neither waits for the other's completion: tensor memory holds
+// two S buffers (S_{j+1} is computed while the softmax works on S_j), a separate
+// bf16 P buffer and the fp32 O accumulator.  Online softmax in base 2 with a lazy
+// running max: O and the row sums are rescaled only when the max grows by more
+// than 2^8; a quarter of the exponentials run on the FMA pipe (exp2_poly).
 // Every wait is bounded; on expiry the CTA drains its in-flight copies/MMAs, frees
 // TMEM and reports kDevErrTimeout through the device error word.
 #include <stdio.h>
@@ -25,11 +31,27 @@
 namespace fva {
 namespace {
 
-constexpr int kAttnThreads = 256;
+#ifdef FVA_ATTN_TRACE
+// Profiling build only: clock64() stamps of pipeline events of CTA 0, by block sequence.
+__device__ unsigned long long g_attn_trace[20][4096];
+#define FVA_TRACE(ev, idx)                                         \
+  do {                                                             \
+    if (blockIdx.x == 0 && (idx) < 4096) g_attn_trace[ev][idx] = clock64(); \
+  } while (0)
+#else
+#define FVA_TRACE(ev, idx) \
+  do {                     \
+  } while (0)
+#endif
+
+constexpr int kAttnThreads = 384;   // 12 warps: 4 control + 8 softmax
 constexpr int kBM = 128;               // MMA M: query rows per tile (S=64 tiles use the top half)
 constexpr float kLazyRescaleLog2 = 8.0f;
+// Of every 8 probabilities a softmax thread computes, this many use the FMA-pipe
+// exp2 (exp2_poly) instead of the MUFU unit, so both units share the work.
+constexpr int kPolyPerEight = 2;
 
-template <int D, int BN, int NS>
+template <int D, int BN, int NSK, int NSV>
 struct AttnCfg {
   static constexpr int NCH = D / 64;                         // 64-column (128-byte) chunks of a row
   static constexpr int Q_CHUNK = kBM * 128;                  // bytes of one Q chunk (128 rows)
@@ -38,15 +60,17 @@ struct AttnCfg {
   static constexpr int KV_BYTES = NCH * KV_CHUNK;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
-  static constexpr int OFF_V = OFF_K + NS * KV_BYTES;
-  static constexpr int OFF_BAR = OFF_V + NS * KV_BYTES;
-  // barriers: q_full, q_empty, o_done, o_free, drain, k_full[NS], v_full[NS], kv_empty[NS], s_full[2], p_full[2]
-  static constexpr int NBAR = 5 + 3 * NS + 4;
-  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;        // tmem base slot, abort flag
-  static constexpr int SMEM = OFF_MISC + 16 + 1024;          // + slack to align the base to 1024
-  static constexpr int TMEM_USED = 2 * BN + D;
-  static constexpr int TMEM_COLS = TMEM_USED <= 32 ? 32 : TMEM_USED <= 64 ? 64 : TMEM_USED <= 128 ? 128
-                                   : TMEM_USED <= 256 ? 256 : 512;
+  static constexpr int OFF_V = OFF_K + NSK * KV_BYTES;
+  static constexpr int OFF_BAR = OFF_V + NSV * KV_BYTES;
+  // barriers: q_full q_empty s_full[2] s_free[2] p_full o_done o_free drain_s drain_pv; k ring; v ring
+  static constexpr int NBAR = 11 + 2 * NSK + 2 * NSV;
+  static constexpr int OFF_RED = OFF_BAR + NBAR * 8;         // row maxima / sums [2 parity][2 half][128]
+  static constexpr int OFF_MISC = OFF_RED + 2 * 2 * kBM * 4; // tmem base slot, abort flag
+  static constexpr int SMEM = OFF_MISC + 16;                 // base must be 1024-aligned (checked)
+  // TMEM columns: S double buffer [0, 2*BN), P [2*BN, 2*BN + BN/2) as bf16 pairs, O after it
+  static constexpr int T_S = 0, T_P = 2 * BN, T_O = 2 * BN + BN / 2;
+  static constexpr int TMEM_USED = T_O + D;
+  static constexpr int TMEM_COLS = TMEM_USED <= 128 ? 128 : TMEM_USED <= 256 ? 256 : 512;
   static constexpr uint32_t IDESC_S = idesc_bf16_f32(kBM, BN, false);
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(kBM, D, true);
   static constexpr uint32_t Q_TX = static_cast<uint32_t>(BN) * D * 2;   // S == BN rows loaded
@@ -76,6 +100,18 @@ __device__ __forceinline__ int item_at(const AttnParams& prm, long long it) {
   }
   return static_cast<int>(u);
 }
+__device__ __forceinline__ int item_count(const AttnParams& prm, int item) {
+  return item < 0 ? 0 : min(prm.counts[item], prm.Nb);
+}
+// Kept key block jj of item `item` (row i), replaced by the diagonal if out of range.
+__device__ __forceinline__ int block_id(const AttnParams& prm, int item, int i, int jj, bool report) {
+  int j = prm.idx[static_cast<long long>(item) * prm.Nb + jj];
+  if (j < 0 || j >= prm.Nb) {
+    if (report) set_device_error(prm.dev_err, kDevErrBadIndex);
+    j = i;
+  }
+  return j;
+}
 
 // Bounded wait that ignores the abort flag (used only while draining).
 __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
@@ -85,24 +121,80 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
   }
 }
 
-template <int D, int BN, int NS>
+// One TMA producer warp: one tile (K or V, 64-column boxes) per kept block through an
+// ns-stage ring; the K producer also loads each item's Q.  The whole warp walks the
+// loop and waits (warp-uniform); lane 0 issues.
+template <int D, int BN, int NS, bool WITH_Q, typename Cfg>
+__device__ void produce(const AttnParams& prm, const CUtensorMap* tm, const CUtensorMap* tmQ, uint32_t ring,
+                        uint32_t full0, uint32_t empty0, uint32_t sQ, uint32_t q_full, uint32_t q_empty,
+                        volatile int* abort_flag) {
+  const int Nb = prm.Nb;
+  const bool leader = (threadIdx.x & 31) == 0;
+  long long g = 0, q_items = 0;
+  bool ok = true;
+  for (long long it = blockIdx.x; it < prm.n_items && ok; it += gridDim.x) {
+    const int item = item_at(prm, it);
+    const int n = item_count(prm, item);
+    if (n <= 0) continue;
+    const long long bh = item / Nb;
+    const int i = item - static_cast<int>(bh * Nb);
+    const long long row0 = bh * prm.N;
+    if (WITH_Q) {
+      if (q_items > 0 && !(ok = __all_sync(0xffffffffu, mbar_wait(q_empty, (q_items - 1) & 1, abort_flag)))) break;
+      if (leader) {
+        mbar_arrive_expect_tx(q_full, Cfg::Q_TX);
+        for (int ch = 0; ch < Cfg::NCH; ++ch)
+          tma_load_2d(sQ + ch * Cfg::Q_CHUNK, tmQ, q_full, ch * 64, static_cast<int>(row0 + static_cast<long long>(i) * BN));
+      }
+      __syncwarp();
+      ++q_items;
+    }
+    for (int jj = 0; jj < n; ++jj, ++g) {
+      const int st = static_cast<int>(g % NS);
+      if (g >= NS && !(ok = __all_sync(0xffffffffu, mbar_wait(empty0 + 8 * st, ((g / NS) - 1) & 1, abort_flag))))
+        break;
+      if (leader) {
+        const int j = block_id(prm, item, i, jj, WITH_Q);
+        mbar_arrive_expect_tx(full0 + 8 * st, Cfg::KV_TX);
+        for (int ch = 0; ch < Cfg::NCH; ++ch)
+          tma_load_2d(ring + st * Cfg::KV_BYTES + ch * Cfg::KV_CHUNK, tm, full0 + 8 * st, ch * 64,
+                      static_cast<int>(row0 + static_cast<long long>(j) * BN));
+      }
+      __syncwarp();
+    }
+  }
+  if (!ok && leader) {
+    // let the copies already issued land before the CTA goes away
+    set_device_error(prm.dev_err, kDevErrTimeout);
+    for (long long q = (g > NS ? g - NS : 0); q < g; ++q) drain_wait(full0 + 8 * (q % NS), (q / NS) & 1);
+    if (WITH_Q && q_items > 0) drain_wait(q_full, (q_items - 1) & 1);
+  }
+  __syncwarp();
+}
+
+template <int D, int BN, int NSK, int NSV>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const AttnParams prm) {
-  using C = AttnCfg<D, BN, NS>;
-  extern __shared__ unsigned char smem_raw[];
-  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  using C = AttnCfg<D, BN, NSK, NSV>;
+  extern __shared__ __align__(1024) unsigned char smem[];
   const uint32_t sbase = smem_u32(smem);
+  if (sbase & 1023u) {
+    // 128-byte-swizzled TMA tiles and MMA operands need 1024-byte alignment
+    if (threadIdx.x == 0) set_device_error(prm.dev_err, kDevErrMisaligned);
+    return;
+  }
   const uint32_t sQ = sbase + C::OFF_Q;
   const uint32_t sK = sbase + C::OFF_K;
   const uint32_t sV = sbase + C::OFF_V;
   const uint32_t bar0 = sbase + C::OFF_BAR;
-  const uint32_t q_full = bar0 + 0, q_empty = bar0 + 8, o_done = bar0 + 16, o_free = bar0 + 24, drain = bar0 + 32;
-  auto k_full = [&](int s) { return bar0 + 40 + 8 * s; };
-  auto v_full = [&](int s) { return bar0 + 40 + 8 * (NS + s); };
-  auto kv_empty = [&](int s) { return bar0 + 40 + 8 * (2 * NS + s); };
-  auto s_full = [&](int b) { return bar0 + 40 + 8 * (3 * NS + b); };
-  auto p_full = [&](int b) { return bar0 + 40 + 8 * (3 * NS + 2 + b); };
+  const uint32_t q_full = bar0, q_empty = bar0 + 8, s_full0 = bar0 + 16, s_free0 = bar0 + 32;
+  const uint32_t p_full = bar0 + 48, o_done = bar0 + 56, o_free = bar0 + 64, drain_s = bar0 + 72;
+  const uint32_t drain_pv = bar0 + 80;
+  const uint32_t k_full0 = bar0 + 88;
+  const uint32_t k_empty0 = k_full0 + 8 * NSK;
+  const uint32_t v_full0 = k_empty0 + 8 * NSK;
+  const uint32_t v_empty0 = v_full0 + 8 * NSV;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -112,17 +204,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
-    mbar_init(o_done, 1);
-    mbar_init(o_free, 128);
-    mbar_init(drain, 1);
-    for (int s = 0; s < NS; ++s) {
-      mbar_init(k_full(s), 1);
-      mbar_init(v_full(s), 1);
-      mbar_init(kv_empty(s), 1);
-    }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(s_full(b), 1);
-      mbar_init(p_full(b), 128);
+      mbar_init(s_full0 + 8 * b, 1);
+      mbar_init(s_free0 + 8 * b, 256);
+    }
+    mbar_init(p_full, 256);
+    mbar_init(o_done, 1);
+    mbar_init(o_free, 256);
+    mbar_init(drain_s, 1);
+    mbar_init(drain_pv, 1);
+    for (int st = 0; st < NSK; ++st) {
+      mbar_init(k_full0 + 8 * st, 1);
+      mbar_init(k_empty0 + 8 * st, 1);
+    }
+    for (int st = 0; st < NSV; ++st) {
+      mbar_init(v_full0 + 8 * st, 1);
+      mbar_init(v_empty0 + 8 * st, 1);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -148,209 +245,235 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS0 = tmem;              // S buffer b at columns b*BN
-  const uint32_t tO = tmem + 2 * BN;      // O accumulator
 
   const long long n_items = prm.n_items;
   const int Nb = prm.Nb;
   const int S = BN;
+  const bool leader = lane == 0;
+  auto wait_all = [&](uint32_t bar, uint32_t parity) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+  };
 
   if (warp == 0) {
-    // ---------------------------------------------------------------- producer
-    if (lane == 0) {
-      long long g = 0;          // running K/V block counter (ring position)
-      long long q_items = 0;    // items whose Q was loaded
-      bool ok = true;
-      for (long long it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-        const int item = item_at(prm, it);
-        const int n = item < 0 ? 0 : min(prm.counts[item], Nb);
-        if (n <= 0) continue;
-        const long long bh = item / Nb;
-        const int i = item - static_cast<int>(bh * Nb);
-        const long long row0 = bh * prm.N;
-        if (q_items > 0 && !(ok = mbar_wait(q_empty, (q_items - 1) & 1, abort_flag))) break;
-        mbar_arrive_expect_tx(q_full, C::Q_TX);
-        for (int ch = 0; ch < C::NCH; ++ch)
-          tma_load_2d(sQ + ch * C::Q_CHUNK, &tmQ, q_full, ch * 64, static_cast<int>(row0 + static_cast<long long>(i) * S));
-        ++q_items;
-        const int32_t* irow = prm.idx + static_cast<long long>(item) * Nb;
-        for (int jj = 0; jj < n; ++jj, ++g) {
-          int j = irow[jj];
-          if (j < 0 || j >= Nb) {
-            set_device_error(prm.dev_err, kDevErrBadIndex);
-            j = i;
-          }
-          const int st = static_cast<int>(g % NS);
-          if (g >= NS && !(ok = mbar_wait(kv_empty(st), ((g / NS) - 1) & 1, abort_flag))) break;
-          const int krow = static_cast<int>(row0 + static_cast<long long>(j) * S);
-          mbar_arrive_expect_tx(k_full(st), C::KV_TX);
+    // ---------------------------------------------------------------- Q + K producer
+    produce<D, BN, NSK, true, C>(prm, &tmK, &tmQ, sK, k_full0, k_empty0, sQ, q_full, q_empty, abort_flag);
+  } else if (warp == 3) {
+    // ---------------------------------------------------------------- V producer
+    produce<D, BN, NSV, false, C>(prm, &tmV, &tmQ, sV, v_full0, v_empty0, sQ, q_full, q_empty, abort_flag);
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- S issuer
+    // S_j = Q K_j^T into S buffer j % 2 once the softmax has read S_{j-2} out of it.
+    // (One thread issues a tcgen05.mma only every ~50 cycles, about the time a
+    // 128x128x16 product takes, so S and PV products come from two warps on
+    // different SM sub-partitions.)  The whole warp walks the loop and waits; lane 0
+    // issues.
+    const uint64_t dQ = sdesc_sw128(sQ, 16, 1024);
+    const uint64_t dK0 = sdesc_sw128(sK, 16, 1024);
+    // (descriptor start addresses are the low 14 bits, address >> 4; operands lie
+    //  below 256 KB, so byte offsets add in without carry)
+    long long g = 0, q_items = 0;
+    bool ok = true, issued = false;
+    for (long long it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+      const int item = item_at(prm, it);
+      const int n = item_count(prm, item);
+      if (n <= 0) continue;
+      if (!(ok = wait_all(q_full, q_items & 1))) break;
+      ++q_items;
+      for (int jj = 0; jj < n; ++jj, ++g) {
+        const int b = static_cast<int>(g & 1);
+        const int st = static_cast<int>(g % NSK);
+        if (g >= 2 && !(ok = wait_all(s_free0 + 8 * b, ((g >> 1) - 1) & 1))) break;
+        if (!(ok = wait_all(k_full0 + 8 * st, (g / NSK) & 1))) break;
+        if (leader) {
+          tc_fence_after();
+          const uint64_t dK = dK0 + static_cast<uint64_t>((st * C::KV_BYTES) >> 4);
+          const uint32_t dS = tmem + C::T_S + b * BN;
+#pragma unroll
           for (int ch = 0; ch < C::NCH; ++ch)
-            tma_load_2d(sK + st * C::KV_BYTES + ch * C::KV_CHUNK, &tmK, k_full(st), ch * 64, krow);
-          mbar_arrive_expect_tx(v_full(st), C::KV_TX);
-          for (int ch = 0; ch < C::NCH; ++ch)
-            tma_load_2d(sV + st * C::KV_BYTES + ch * C::KV_CHUNK, &tmV, v_full(st), ch * 64, krow);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_ss(dS, dQ + ((ch * C::Q_CHUNK + kk * 32) >> 4), dK + ((ch * C::KV_CHUNK + kk * 32) >> 4),
+                      C::IDESC_S, (ch | kk) != 0);
+          umma_commit(k_empty0 + 8 * st);
+          umma_commit(s_full0 + 8 * b);
+          if (jj == n - 1) umma_commit(q_empty);   // last reader of this item's Q
         }
-      }
-      if (!ok) {
-        // let the copies already issued land before the CTA goes away
-        set_device_error(prm.dev_err, kDevErrTimeout);
-        for (long long q = (g > NS ? g - NS : 0); q < g; ++q) {
-          const int st = static_cast<int>(q % NS);
-          drain_wait(k_full(st), (q / NS) & 1);
-          drain_wait(v_full(st), (q / NS) & 1);
-        }
-        if (q_items > 0) drain_wait(q_full, (q_items - 1) & 1);
+        __syncwarp();
+        issued = true;
       }
     }
-  } else if (warp == 1) {
-    // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      long long g = 0;          // K/V ring position (same sequence as the producer)
-      long long sidx = 0;       // S buffer sequence number
-      long long q_items = 0, o_items = 0;
-      bool ok = true;
-      bool issued = false;
-      for (long long it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-        const int item = item_at(prm, it);
-        const int n = item < 0 ? 0 : min(prm.counts[item], Nb);
-        if (n <= 0) continue;
-        if (!(ok = mbar_wait(q_full, q_items & 1, abort_flag))) break;
-        ++q_items;
-        // S_jj = Q K_jj^T into S buffer (sidx + jj) & 1
-        auto issue_s = [&](int jj) -> bool {
-          const long long gg = g + jj;
-          const int st = static_cast<int>(gg % NS);
-          if (!mbar_wait(k_full(st), (gg / NS) & 1, abort_flag)) return false;
+    if (!ok && leader) set_device_error(prm.dev_err, kDevErrTimeout);
+    if (issued) {
+      if (leader) umma_commit(drain_s);
+      __syncwarp();
+      drain_wait(drain_s, 0);
+    }
+  } else if (warp == 2) {
+    // ---------------------------------------------------------------- PV issuer
+    // O += P_j V_j once the softmax has written P_j (p_full).
+    const uint64_t dV0 = sdesc_sw128(sV, C::KV_CHUNK, 1024);
+    long long g = 0, items = 0;
+    bool ok = true, issued = false;
+    for (long long it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+      const int item = item_at(prm, it);
+      const int n = item_count(prm, item);
+      if (n <= 0) continue;
+      if (items > 0 && !(ok = wait_all(o_free, (items - 1) & 1))) break;   // epilogue read O
+      for (int jj = 0; jj < n; ++jj, ++g) {
+        const int st = static_cast<int>(g % NSV);
+        if (!(ok = wait_all(p_full, g & 1))) break;
+        if (!(ok = wait_all(v_full0 + 8 * st, (g / NSV) & 1))) break;
+        if (leader) {
           tc_fence_after();
-          const uint32_t dS = tS0 + static_cast<uint32_t>(((sidx + jj) & 1) * BN);
+          const uint64_t dV = dV0 + static_cast<uint64_t>((st * C::KV_BYTES) >> 4);
+          const uint32_t aP = tmem + C::T_P;
 #pragma unroll
-          for (int ch = 0; ch < C::NCH; ++ch)
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t ad = sdesc_sw128(sQ + ch * C::Q_CHUNK + kk * 32, 16, 1024);
-              const uint64_t bd = sdesc_sw128(sK + st * C::KV_BYTES + ch * C::KV_CHUNK + kk * 32, 16, 1024);
-              umma_ss(dS, ad, bd, C::IDESC_S, (ch | kk) != 0);
-            }
-          umma_commit(s_full(static_cast<int>((sidx + jj) & 1)));
-          issued = true;
-          if (jj == n - 1) umma_commit(q_empty);   // last reader of this item's Q
-          return true;
-        };
-        if (!(ok = issue_s(0))) break;
-        for (int jj = 0; jj < n; ++jj) {
-          if (jj + 1 < n && !(ok = issue_s(jj + 1))) break;
-          const long long gg = g + jj;
-          const int st = static_cast<int>(gg % NS);
-          const int sb = static_cast<int>((sidx + jj) & 1);
-          if (jj == 0 && o_items > 0 && !(ok = mbar_wait(o_free, (o_items - 1) & 1, abort_flag))) break;
-          if (!(ok = mbar_wait(p_full(sb), ((sidx + jj) >> 1) & 1, abort_flag))) break;
-          if (!(ok = mbar_wait(v_full(st), (gg / NS) & 1, abort_flag))) break;
-          tc_fence_after();
-          const uint32_t aP = tS0 + static_cast<uint32_t>(sb * BN);
-#pragma unroll
-          for (int ks = 0; ks < BN / 16; ++ks) {
-            const uint64_t bd = sdesc_sw128(sV + st * C::KV_BYTES + ks * 16 * 128, C::KV_CHUNK, 1024);
-            umma_ts(tO, aP + ks * 8, bd, C::IDESC_PV, (jj > 0 || ks > 0) ? 1u : 0u);
-          }
-          umma_commit(kv_empty(st));
+          for (int ks = 0; ks < BN / 16; ++ks)
+            umma_ts(tmem + C::T_O, aP + ks * 8, dV + ((ks * 16 * 128) >> 4), C::IDESC_PV,
+                    (jj > 0 || ks > 0) ? 1u : 0u);
+          umma_commit(v_empty0 + 8 * st);
           umma_commit(o_done);
         }
-        if (!ok) break;
-        g += n;
-        sidx += n;
-        ++o_items;
+        __syncwarp();
+        issued = true;
       }
-      if (!ok) set_device_error(prm.dev_err, kDevErrTimeout);
-      if (issued) {
-        // every MMA issued by this thread has completed before TMEM is released
-        umma_commit(drain);
-        drain_wait(drain, 0);
-      }
+      ++items;
+    }
+    if (!ok && leader) set_device_error(prm.dev_err, kDevErrTimeout);
+    if (issued) {
+      if (leader) umma_commit(drain_pv);
+      __syncwarp();
+      drain_wait(drain_pv, 0);
     }
   } else if (warp >= 4) {
     // ---------------------------------------------------------------- softmax
-    // (waits are made warp-uniform: the tcgen05.ld/st below are warp-collective)
-    const int row = (warp - 4) * 32 + lane;                      // TMEM lane == query row
-    const uint32_t lane_off = static_cast<uint32_t>((warp - 4) * 32) << 16;
+    // Eight warps: warp w owns TMEM lane quarter w % 4 (query rows 32*(w%4) ...) and
+    // half h = (w - 4) / 4 of the columns of S (and of P and O).  The two warps of a
+    // quarter meet at named barrier 1 + quarter once per block to combine their row
+    // maxima (and twice per item for the row sums); the barrier also ANDs their
+    // "still ok" flags so a bounded-wait failure makes both leave together.  Waits
+    // are warp-uniform: the tcgen05.ld/st below are warp-collective.
+    constexpr int HB = BN / 2;                                    // S columns per half
+    constexpr int HD = D / 2;                                     // O columns per half
+    const int quarter = warp & 3;
+    const int half = (warp - 4) >> 2;
+    const int row = quarter * 32 + lane;                          // TMEM lane == query row
+    const int pair_bar = 1 + quarter;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tP = tmem + C::T_P + half * (HB / 2) + lane_off;
+    const uint32_t tO = tmem + C::T_O + half * HD + lane_off;
+    float* red_max = reinterpret_cast<float*>(smem + C::OFF_RED);         // [2][2][kBM]
     const float sl2 = prm.scale_log2;
-    long long sidx = 0, o_cnt = 0;
+    long long g = 0, o_cnt = 0;    // blocks processed; o_done phases observed
     bool ok = true;
+    // observe o_done phases up to `upto` (the PV products of blocks <= upto are done)
+    auto need_o = [&](long long upto) {
+      while (ok && o_cnt <= upto) {
+        ok = __all_sync(0xffffffffu, mbar_wait(o_done, o_cnt & 1, abort_flag));
+        ++o_cnt;
+      }
+    };
     for (long long it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
       const int item = item_at(prm, it);
       if (item < 0) continue;
-      const int n = min(prm.counts[item], Nb);
+      const int n = item_count(prm, item);
       const long long bh = item / Nb;
       const int i = item - static_cast<int>(bh * Nb);
-      uint16_t* orow = prm.out + (bh * prm.N + static_cast<long long>(i) * S + row) * D;
+      uint16_t* orow = prm.out + (bh * prm.N + static_cast<long long>(i) * S + row) * D + half * HD;
       if (n <= 0) {
         if (row < S)
-          for (int c = 0; c < D; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
+          for (int c = 0; c < HD; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
         continue;
       }
-      float m = -INFINITY;   // running max of the scaled logits (base-2 units)
-      float l = 0.0f;        // running row sum at max m
-      for (int jj = 0; jj < n; ++jj) {
-        const int sb = static_cast<int>((sidx + jj) & 1);
-        ok = __all_sync(0xffffffffu, mbar_wait(s_full(sb), ((sidx + jj) >> 1) & 1, abort_flag));
+      float m = -INFINITY;   // running max of the scaled logits (base-2 units), same in both halves
+      float l = 0.0f;        // this half's running row sum at max m
+      for (int jj = 0; jj < n; ++jj, ++g) {
+        const int b = static_cast<int>(g & 1);
+        const int par = b;
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(s_full0 + 8 * b, (g >> 1) & 1, abort_flag));
+        uint32_t r[HB];
+        float pm = -INFINITY;
+        if (ok) {
+          tc_fence_after();
+          const uint32_t tS = tmem + C::T_S + b * BN + half * HB + lane_off;
+#pragma unroll
+          for (int c = 0; c < HB / 32; ++c) tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
+          tmem_wait_ld();
+          tc_fence_before();
+          mbar_arrive(s_free0 + 8 * b);                           // S_j read out: buffer b may be refilled
+          float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+          for (int c = 0; c < HB; c += 4) {
+            mx[0] = fmax3(mx[0], __uint_as_float(r[c]), __uint_as_float(r[c + 1]));
+            mx[1] = fmax3(mx[1], __uint_as_float(r[c + 2]), __uint_as_float(r[c + 3]));
+          }
+          pm = fmaxf(mx[0], mx[1]);
+          red_max[(par * 2 + half) * kBM + row] = pm;
+        }
+        ok = bar_and(pair_bar, 64, ok);                           // both halves' maxima published
         if (!ok) break;
-        tc_fence_after();
-        uint32_t r[BN];
-        const uint32_t tS = tS0 + static_cast<uint32_t>(sb * BN) + lane_off;
-#pragma unroll
-        for (int c = 0; c < BN / 32; ++c) tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
-        tmem_wait_ld();
-        float mx = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < BN; ++c) mx = fmaxf(mx, __uint_as_float(r[c]));
-        const float m_cand = mx * sl2;
+        const float m_cand = fmaxf(pm, red_max[(par * 2 + (half ^ 1)) * kBM + row]) * sl2;
         float alpha = 1.0f;
         if (m_cand > m + kLazyRescaleLog2) {
           alpha = ex2_approx(m - m_cand);   // 0 on the first block (m = -inf)
           m = m_cand;
         }
-        float rs = 0.0f;
+        float rs[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-        for (int c = 0; c < BN / 2; ++c) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(r[2 * c]), sl2, -m));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(r[2 * c + 1]), sl2, -m));
-          rs += p0 + p1;
+        for (int c = 0; c < HB / 2; ++c) {
+          const float x0 = fmaf(__uint_as_float(r[2 * c]), sl2, -m);
+          const float x1 = fmaf(__uint_as_float(r[2 * c + 1]), sl2, -m);
+          const bool poly = (c % 4) < (kPolyPerEight / 2);
+          const float p0 = poly ? exp2_poly(x0) : ex2_approx(x0);
+          const float p1 = poly ? exp2_poly(x1) : ex2_approx(x1);
+          rs[(2 * c) & 3] += p0;
+          rs[(2 * c + 1) & 3] += p1;
           r[c] = pack_bf16x2(p0, p1);
         }
-        l = l * alpha + rs;
-#pragma unroll
-        for (int c = 0; c < BN / 64; ++c) tmem_st32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
-        if (jj > 0) {
-          // O must hold P_{jj-1} V_{jj-1} before it is rescaled and P_jj V_jj is added
-          ok = __all_sync(0xffffffffu, mbar_wait(o_done, o_cnt & 1, abort_flag));
-          if (!ok) break;
-          ++o_cnt;
+        l = l * alpha + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
+        // P and O are read / written by P_{g-1} V_{g-1}: wait for it before touching them
+        need_o(g - 1);
+        if (ok) {
           tc_fence_after();
-          if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+          if constexpr (HB / 2 >= 32) {
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
+            for (int c = 0; c < HB / 64; ++c) tmem_st32(tP + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
+          } else {
+            tmem_st16(tP, r);
+          }
+          if (jj > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+#pragma unroll
+            for (int c = 0; c < HD / 32; ++c) {
               uint32_t o[32];
-              tmem_ld32(tO + lane_off + c * 32, o);
+              tmem_ld32(tO + c * 32, o);
               tmem_wait_ld();
 #pragma unroll
               for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-              tmem_st32(tO + lane_off + c * 32, o);
+              tmem_st32(tO + c * 32, o);
             }
           }
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(p_full);
         }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(p_full(sb));
       }
+      // no early exit before these barriers: the partner warp must meet them too.  The
+      // row sums go through the parity region the next block will use; both warps
+      // are past their last reads of it, and the second barrier keeps the next
+      // block's maxima from overwriting it before both have read it.
+      need_o(g - 1);
+      float* red_l = red_max + (g & 1) * 2 * kBM;
+      red_l[half * kBM + row] = l;
+      ok = bar_and(pair_bar, 64, ok);
       if (!ok) break;
-      ok = __all_sync(0xffffffffu, mbar_wait(o_done, o_cnt & 1, abort_flag));
+      const float inv = 1.0f / (red_l[row] + red_l[kBM + row]);
+      ok = bar_and(pair_bar, 64, ok);
       if (!ok) break;
-      ++o_cnt;
       tc_fence_after();
-      const float inv = 1.0f / l;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < HD / 32; ++c) {
         uint32_t o[32];
-        tmem_ld32(tO + lane_off + c * 32, o);
+        tmem_ld32(tO + c * 32, o);
         tmem_wait_ld();
         uint32_t pk[16];
 #pragma unroll
@@ -364,7 +487,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       tc_fence_before();
       mbar_arrive(o_free);
-      sidx += n;
     }
     if (!ok) set_device_error(prm.dev_err, kDevErrTimeout);
   }
@@ -424,15 +546,17 @@ int sm_count() {
   return n;
 }
 
-template <int D, int BN, int NS>
+template <int D, int BN, int NSK, int NSV>
 cudaError_t launch_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const AttnParams& prm,
                      cudaStream_t s) {
-  using C = AttnCfg<D, BN, NS>;
+  using C = AttnCfg<D, BN, NSK, NSV>;
   static_assert(C::SMEM <= 232448, "shared memory budget");
-  cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, BN, NS>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  static_assert(C::TMEM_USED <= 512, "tensor memory budget");
+  cudaError_t e =
+      cudaFuncSetAttribute(attn_kernel<D, BN, NSK, NSV>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   const long long grid = prm.n_items < sm_count() ? prm.n_items : sm_count();
-  attn_kernel<D, BN, NS><<<static_cast<unsigned>(grid), kAttnThreads, C::SMEM, s>>>(mq, mk, mv, prm);
+  attn_kernel<D, BN, NSK, NSV><<<static_cast<unsigned>(grid), kAttnThreads, C::SMEM, s>>>(mq, mk, mv, prm);
   return cudaGetLastError();
 }
 
@@ -458,15 +582,21 @@ cudaError_t launch_attention(const void* qr, const void* kr, const void* vr, con
   prm.scale_log2 = scale * 1.4426950408889634f;
   cudaError_t e;
   if (D.d == 128 && D.S == 128)
-    e = launch_t<128, 128, 2>(mq, mk, mv, prm, s);
+    e = launch_t<128, 128, 3, 3>(mq, mk, mv, prm, s);
   else if (D.d == 128 && D.S == 64)
-    e = launch_t<128, 64, 4>(mq, mk, mv, prm, s);
+    e = launch_t<128, 64, 5, 5>(mq, mk, mv, prm, s);
   else if (D.d == 64 && D.S == 128)
-    e = launch_t<64, 128, 4>(mq, mk, mv, prm, s);
+    e = launch_t<64, 128, 5, 5>(mq, mk, mv, prm, s);
   else
-    e = launch_t<64, 64, 4>(mq, mk, mv, prm, s);
+    e = launch_t<64, 64, 6, 6>(mq, mk, mv, prm, s);
   ++*launches;
   return e;
 }
 
 }  // namespace fva
+
+#ifdef FVA_ATTN_TRACE
+extern "C" int fva_debug_attn_trace(unsigned long long* host_out) {
+  return cudaMemcpyFromSymbol(host_out, fva::g_attn_trace, sizeof(fva::g_attn_trace)) == cudaSuccess ? 0 : 3;
+}
+#endif

@@ -13,6 +13,7 @@ enum : int {
   kDevErrNone = 0,
   kDevErrTimeout = 1,      // a bounded wait on an mbarrier expired
   kDevErrBadIndex = 2,     // a key-block id outside [0, Nb) was found in a list
+  kDevErrMisaligned = 3,   // dynamic shared memory was not 1024-byte aligned
 };
 
 // Roughly 2 s at 1.9 GHz: no single pipeline wait in these kernels is anywhere near it.
@@ -165,6 +166,78 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Base-2 exponential on the FMA/ALU pipes (no MUFU or conversion unit), for
+// x <= 2^7; inputs below -125 give ~2^-125.  Cody-Waite style range reduction
+// x = n + f with n = round-to-nearest(x) taken from the low mantissa bits of
+// x + 1.5*2^23, f in [-0.5, 0.5]; a cubic gives 2^f and n is added to its exponent
+// field (the shifted sum's high bits carry n << 23 modulo 2^32).  The cubic is our
+// own least-squares fit of 2^f on Chebyshev nodes of [-0.5, 0.5] with relative-error
+// weighting, iteratively reweighted towards equal ripple: max relative error 7.5e-5,
+// far below the 2^-9 relative step of the bfloat16 probabilities it feeds.  Its value
+// lies in [0.70, 1.42], so the exponent field is 126 or 127 and n >= -125 keeps the
+// sum a positive normal number.
+constexpr float kExp2C0 = 0.9999280571937561f;
+constexpr float kExp2C1 = 0.6932609677314758f;
+constexpr float kExp2C2 = 0.2426111251115799f;
+constexpr float kExp2C3 = 0.05517163127660751f;
+constexpr float kRoundMagic = 12582912.0f;   // 1.5 * 2^23
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -125.0f);
+  const float t = x + kRoundMagic;
+  const float f = x - (t - kRoundMagic);
+  const float p = fmaf(fmaf(fmaf(kExp2C3, f, kExp2C2), f, kExp2C1), f, kExp2C0);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// Packed fp32 pairs (sm_100): two lanes of work per instruction.
+__device__ __forceinline__ uint64_t f32x2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f32x2_unpack(uint64_t r, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(r));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// AND of `pred` over the `nthreads` threads (whole warps) that meet at named barrier `id`.
+__device__ __forceinline__ bool bar_and(int id, int nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %1, 0;\n\t"
+      "bar.red.and.pred po, %2, %3, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}\n"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
+}
+
+// 32 lanes x 16 columns store (half of tmem_st32).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
