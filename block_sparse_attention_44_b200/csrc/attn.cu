@@ -62,8 +62,8 @@ struct AttnCfg {
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
   static constexpr int OFF_V = OFF_K + NSK * KV_BYTES;
   static constexpr int OFF_BAR = OFF_V + NSV * KV_BYTES;
-  // barriers: q_full q_empty s_full[2] s_free[2] p_full o_done o_free drain_s drain_pv; k ring; v ring
-  static constexpr int NBAR = 11 + 2 * NSK + 2 * NSV;
+  // barriers: q_full q_empty s_full[2] s_free[2] p_full[2] o_done o_free drain_s drain_pv; k ring; v ring
+  static constexpr int NBAR = 12 + 2 * NSK + 2 * NSV;
   static constexpr int OFF_RED = OFF_BAR + NBAR * 8;         // row maxima / sums [2 parity][2 half][128]
   static constexpr int OFF_MISC = OFF_RED + 2 * 2 * kBM * 4; // tmem base slot, abort flag
   static constexpr int SMEM = OFF_MISC + 16;                 // base must be 1024-aligned (checked)
@@ -189,9 +189,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t sV = sbase + C::OFF_V;
   const uint32_t bar0 = sbase + C::OFF_BAR;
   const uint32_t q_full = bar0, q_empty = bar0 + 8, s_full0 = bar0 + 16, s_free0 = bar0 + 32;
-  const uint32_t p_full = bar0 + 48, o_done = bar0 + 56, o_free = bar0 + 64, drain_s = bar0 + 72;
-  const uint32_t drain_pv = bar0 + 80;
-  const uint32_t k_full0 = bar0 + 88;
+  const uint32_t p_full0 = bar0 + 48, o_done = bar0 + 64, o_free = bar0 + 72, drain_s = bar0 + 80;
+  const uint32_t drain_pv = bar0 + 88;
+  const uint32_t k_full0 = bar0 + 96;
   const uint32_t k_empty0 = k_full0 + 8 * NSK;
   const uint32_t v_full0 = k_empty0 + 8 * NSK;
   const uint32_t v_empty0 = v_full0 + 8 * NSV;
@@ -207,8 +207,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(s_full0 + 8 * b, 1);
       mbar_init(s_free0 + 8 * b, 256);
+      mbar_init(p_full0 + 8 * b, 256);
     }
-    mbar_init(p_full, 256);
     mbar_init(o_done, 1);
     mbar_init(o_free, 256);
     mbar_init(drain_s, 1);
@@ -282,8 +282,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       for (int jj = 0; jj < n; ++jj, ++g) {
         const int b = static_cast<int>(g & 1);
         const int st = static_cast<int>(g % NSK);
-        if (g >= 2 && !(ok = wait_all(s_free0 + 8 * b, ((g >> 1) - 1) & 1))) break;
+        // S_g is issued when the softmax hands over P_{g-2} (buffer b is free by then, and
+        // P_{g-2} V_{g-2} is issued at the same moment): running S further ahead would
+        // only queue it in front of the PV product the softmax waits on
+        if (g >= 2 && !(ok = wait_all(p_full0 + 8 * b, ((g >> 1) - 1) & 1))) break;
+        if (leader) FVA_TRACE(4, g);
         if (!(ok = wait_all(k_full0 + 8 * st, (g / NSK) & 1))) break;
+        if (leader) FVA_TRACE(9, g);
         if (leader) {
           tc_fence_after();
           const uint64_t dK = dK0 + static_cast<uint64_t>((st * C::KV_BYTES) >> 4);
@@ -297,6 +302,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           umma_commit(k_empty0 + 8 * st);
           umma_commit(s_full0 + 8 * b);
           if (jj == n - 1) umma_commit(q_empty);   // last reader of this item's Q
+          FVA_TRACE(5, g);
         }
         __syncwarp();
         issued = true;
@@ -321,8 +327,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (items > 0 && !(ok = wait_all(o_free, (items - 1) & 1))) break;   // epilogue read O
       for (int jj = 0; jj < n; ++jj, ++g) {
         const int st = static_cast<int>(g % NSV);
-        if (!(ok = wait_all(p_full, g & 1))) break;
+        if (!(ok = wait_all(p_full0 + 8 * static_cast<int>(g & 1), (g >> 1) & 1))) break;
+        if (leader) FVA_TRACE(6, g);
         if (!(ok = wait_all(v_full0 + 8 * st, (g / NSV) & 1))) break;
+        if (leader) FVA_TRACE(10, g);
         if (leader) {
           tc_fence_after();
           const uint64_t dV = dV0 + static_cast<uint64_t>((st * C::KV_BYTES) >> 4);
@@ -333,6 +341,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     (jj > 0 || ks > 0) ? 1u : 0u);
           umma_commit(v_empty0 + 8 * st);
           umma_commit(o_done);
+          FVA_TRACE(7, g);
         }
         __syncwarp();
         issued = true;
@@ -364,6 +373,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint32_t tO = tmem + C::T_O + half * HD + lane_off;
     float* red_max = reinterpret_cast<float*>(smem + C::OFF_RED);         // [2][2][kBM]
     const float sl2 = prm.scale_log2;
+    const uint64_t sl2x2 = f32x2_pack(sl2, sl2);
     long long g = 0, o_cnt = 0;    // blocks processed; o_done phases observed
     bool ok = true;
     // observe o_done phases up to `upto` (the PV products of blocks <= upto are done)
@@ -391,6 +401,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int b = static_cast<int>(g & 1);
         const int par = b;
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(s_full0 + 8 * b, (g >> 1) & 1, abort_flag));
+        if (warp == 4 && lane == 0) FVA_TRACE(0, g);
         uint32_t r[HB];
         float pm = -INFINITY;
         if (ok) {
@@ -412,27 +423,34 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         ok = bar_and(pair_bar, 64, ok);                           // both halves' maxima published
         if (!ok) break;
+        if (warp == 4 && lane == 0) FVA_TRACE(1, g);
         const float m_cand = fmaxf(pm, red_max[(par * 2 + (half ^ 1)) * kBM + row]) * sl2;
         float alpha = 1.0f;
         if (m_cand > m + kLazyRescaleLog2) {
           alpha = ex2_approx(m - m_cand);   // 0 on the first block (m = -inf)
           m = m_cand;
         }
-        float rs[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        const uint64_t negm = f32x2_pack(-m, -m);
+        uint64_t rs[4] = {0, 0, 0, 0};      // packed partial row sums
 #pragma unroll
         for (int c = 0; c < HB / 2; ++c) {
-          const float x0 = fmaf(__uint_as_float(r[2 * c]), sl2, -m);
-          const float x1 = fmaf(__uint_as_float(r[2 * c + 1]), sl2, -m);
+          // x = s * scale_log2 - m for two columns at once
+          const uint64_t x2 = ffma2(f32x2_pack(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1])), sl2x2, negm);
+          float x0, x1;
+          f32x2_unpack(x2, x0, x1);
           const bool poly = (c % 4) < (kPolyPerEight / 2);
           const float p0 = poly ? exp2_poly(x0) : ex2_approx(x0);
           const float p1 = poly ? exp2_poly(x1) : ex2_approx(x1);
-          rs[(2 * c) & 3] += p0;
-          rs[(2 * c + 1) & 3] += p1;
+          rs[c & 3] = fadd2(rs[c & 3], f32x2_pack(p0, p1));
           r[c] = pack_bf16x2(p0, p1);
         }
-        l = l * alpha + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
+        float a0, a1;
+        f32x2_unpack(fadd2(fadd2(rs[0], rs[1]), fadd2(rs[2], rs[3])), a0, a1);
+        l = l * alpha + (a0 + a1);
+        if (warp == 4 && lane == 0) FVA_TRACE(2, g);
         // P and O are read / written by P_{g-1} V_{g-1}: wait for it before touching them
         need_o(g - 1);
+        if (warp == 4 && lane == 0) FVA_TRACE(8, g);
         if (ok) {
           tc_fence_after();
           if constexpr (HB / 2 >= 32) {
@@ -454,7 +472,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
           tmem_wait_st();
           tc_fence_before();
-          mbar_arrive(p_full);
+          mbar_arrive(p_full0 + 8 * b);
+          if (warp == 4 && lane == 0) FVA_TRACE(3, g);
         }
       }
       // no early exit before these barriers: the partner warp must meet them too.  The
