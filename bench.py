@@ -48,6 +48,9 @@ def parse():
     ap.add_argument("--impl", default="fva", choices=["fva", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--static-order", action="store_true", help="item-id order instead of the LPT work list")
+    ap.add_argument("--report", choices=["stress", "sweep"], default=None,
+                    help="instead of the headline line: head-heterogeneity stress (LPT vs item-id order) or the "
+                         "p x tile sweep at 720p scale, one JSON line per measurement")
     return ap.parse_args()
 
 
@@ -380,6 +383,83 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ reports ----------
+def _time_ms(fn, stream, reps):
+    import torch
+    E = lambda: torch.cuda.Event(enable_timing=True)
+    a, b = E(), E()
+    fn()
+    torch.cuda.synchronize()
+    a.record(stream)
+    for _ in range(reps):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / reps
+
+
+def cta_imbalance(counts, order, n_cta):
+    """lambda_SM = max / mean kept block pairs per CTA when CTAs stride through `order`."""
+    per = np.zeros(n_cta)
+    for pos, u in enumerate(order):
+        per[pos % n_cta] += counts[u]
+    return float(per.max() / per.mean())
+
+
+def run_report(args):
+    import torch
+    import block_sparse_attention_44_b200 as fva
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream(dev)
+    n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
+    peaks = load_peaks()
+    base = synth.CONFIGS["stress720p" if args.report == "stress" else "wan720p"]
+    q, k, v = synth.make_qkv(base)
+    def host_bf16(a):
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+    qd, kd, vd = host_bf16(q), host_bf16(k), host_bf16(v)
+    del q, k, v
+    if args.report == "stress":
+        cases = [base]
+    else:
+        cases = [c for c in synth.sweep_configs()]
+    for cfg in cases:
+        g = fva.Geom.of(cfg)
+        path = fva.SparseAttention(g, cfg.p, cfg.k, device=dev)
+        out = torch.empty_like(qd)
+        path(qd, kd, vd, out, stream)
+        torch.cuda.synchronize()
+        assert fva.fva_get_device_error(stream) == 0
+        counts = path.rep.counts.cpu().numpy().reshape(-1)
+        pairs = int(counts.sum())
+        flops = 4.0 * g.S * g.S * g.d * pairs
+        dense = 4.0 * g.B * g.H * float(g.N) ** 2 * g.d
+        route_ms = _time_ms(lambda: path.routing(stream), stream, 5)
+        path.use_lpt = True
+        lpt_ms = _time_ms(lambda: path.attention(stream), stream, 5)
+        line = {"report": args.report, "workload": cfg.name, "tile": g.S, "blocks": g.Nb, "p": cfg.p, "k": cfg.k,
+                "density": pairs / float(g.B * g.H * g.Nb * g.Nb),
+                "attn_ms": lpt_ms, "attn_tflops": flops / (lpt_ms * 1e-3) / 1e12,
+                "attn_dense_equiv_tflops": dense / (lpt_ms * 1e-3) / 1e12,
+                "attn_frac_sustained_peak": flops / (lpt_ms * 1e-3) / 1e12 / peaks["bf16_tflops_sustained"],
+                "route_repair_ms": route_ms, "routing_gbs": 2.0 * g.B * g.H * g.N * g.d * 2 / (route_ms * 1e-3) / 1e9,
+                "routing_overhead_pct": 100.0 * route_ms / lpt_ms}
+        if args.report == "stress":
+            wl = path.rep.worklist.cpu().numpy()
+            hw = path.rep.head_work.cpu().numpy().reshape(-1)
+            path.use_lpt = False
+            static_ms = _time_ms(lambda: path.attention(stream), stream, 5)
+            path.use_lpt = True
+            line.update({"static_order_attn_ms": static_ms, "lpt_speedup": static_ms / lpt_ms,
+                         "lambda_sm_lpt": cta_imbalance(counts, wl, n_sm),
+                         "lambda_sm_static": cta_imbalance(counts, np.arange(counts.size), n_sm),
+                         "head_density_even": float(hw[0::2].mean() / (g.Nb * g.Nb)),
+                         "head_density_odd": float(hw[1::2].mean() / (g.Nb * g.Nb))})
+        print(json.dumps(line), flush=True)
+        del path, out
+        torch.cuda.empty_cache()
+
+
 def main():
     args = parse()
     rank = int(os.environ.get("RANK", "0"))
@@ -387,6 +467,9 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.report:
+        run_report(args)
         return
     import torch
     import torch.distributed as dist
