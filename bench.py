@@ -268,7 +268,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
     # --- timed region: K whole steps; per-stage events on the launching stream
     K = args.steps
     E = lambda: torch.cuda.Event(enable_timing=True)
-    ev = [[E() for _ in range(6)] for _ in range(K)]
+    ev = [[E() for _ in range(5)] for _ in range(K)]
     gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
     if world > 1:
         dist.barrier()
@@ -284,16 +284,12 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
             fva.fva_reorder(kd, path.kr, g, stream)
             fva.fva_reorder(vd, path.vr, g, stream)
             e[1].record(stream)
-            fva.fva_route(path.qr, path.kr, g, cfg.p, cfg.k, path.route.topp_mask, path.route.topk_idx, path.ws,
-                          stream=stream)
+            path.routing(stream)                  # fva_route_repair: route + repair + LPT list
             e[2].record(stream)
-            fva.fva_repair(path.route.topp_mask, path.route.topk_idx, g, cfg.k, path.rep.counts, path.rep.idx,
-                           path.rep.head_work, path.rep.worklist, stream=stream)
-            e[3].record(stream)
             path.attention(stream)
-            e[4].record(stream)
+            e[3].record(stream)
             fva.fva_inverse_reorder(path.outr, out, g, stream)
-            e[5].record(stream)
+            e[4].record(stream)
         stop.record(stream)
         torch.cuda.synchronize(dev)
     launches = fva.fva_launch_count() - launches0
@@ -304,10 +300,18 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         total_ms = float(t.item())
     ms = total_ms / K
-    stage = np.array([[ev[s][i].elapsed_time(ev[s][i + 1]) for i in range(5)] for s in range(K)])
-    st_mean = stage.mean(axis=0)            # reorder x3, route, repair, attention, inverse (ms)
-    attn_ms = float(st_mean[3])
-    route_ms = float(st_mean[1] + st_mean[2])
+    stage = np.array([[ev[s][i].elapsed_time(ev[s][i + 1]) for i in range(4)] for s in range(K)])
+    st_mean = stage.mean(axis=0)            # reorder x3, route + repair (fused), attention, inverse (ms)
+    attn_ms = float(st_mean[2])
+    route_ms = float(st_mean[1])
+
+    # the unfused entry points, timed apart (same inputs): fva_route, then fva_repair
+    sep_route_ms = _time_ms(lambda: fva.fva_route(path.qr, path.kr, g, cfg.p, cfg.k, path.route.topp_mask,
+                                                  path.route.topk_idx, path.ws, stream=stream), stream, 10)
+    sep_repair_ms = _time_ms(lambda: fva.fva_repair(path.route.topp_mask, path.route.topk_idx, g, cfg.k,
+                                                    path.rep.counts, path.rep.idx, path.rep.head_work,
+                                                    path.rep.worklist, stream=stream), stream, 10)
+    path.routing(stream)
 
     # --- end to end through host buffers (pinned H2D of Q/K/V, the path, D2H of O)
     h2d = 3 * qh.numel() * 2
@@ -364,8 +368,9 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
         "routing_frac_hbm": bytes_route / (route_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
         "reorder_gbs": bytes_reorder / (st_mean[0] * 1e-3) / 1e9,
         "routing_overhead_pct": 100.0 * route_ms / attn_ms,
-        "stage_ms": {"reorder_qkv": st_mean[0], "route": st_mean[1], "repair": st_mean[2], "attention": st_mean[3],
-                     "inverse_reorder": st_mean[4]},
+        "stage_ms": {"reorder_qkv": st_mean[0], "route_repair_fused": st_mean[1], "attention": st_mean[2],
+                     "inverse_reorder": st_mean[3], "route_unfused": sep_route_ms, "repair_unfused": sep_repair_ms},
+        "routing_unfused_gbs": bytes_route / ((sep_route_ms + sep_repair_ms) * 1e-3) / 1e9,
         "roofline": {"bound": "tensor", "kernel": "attn_kernel (fva_block_sparse_attn)", "achieved": achieved,
                      "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                      "peak_src": f"{peaks['src']} bf16 sustained (kernel timed inside a long step loop)",

@@ -83,6 +83,7 @@ def _load():
         "fva_route_workspace_size": ([_Geom], sz),
         "fva_route": ([vp, vp, _Geom, f64, i32, vp, vp, vp, vp, sz, vp], ctypes.c_int),
         "fva_route_static": ([vp, vp, _Geom, f64, i32, vp, vp, vp, vp], ctypes.c_int),
+        "fva_route_repair": ([vp, vp, _Geom, f64, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
         "fva_repair_workspace_size": ([_Geom], sz),
         "fva_repair": ([vp, vp, _Geom, i32, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
         "fva_block_sparse_attn": ([vp, vp, vp, vp, vp, vp, _Geom, f32, vp, vp], ctypes.c_int),
@@ -183,6 +184,26 @@ def fva_route_static(qr, kr, g: Geom, p: float, k: int, topp_mask, topk_idx, log
                                 _ptr(logits_out), _stream(stream)))
 
 
+def fva_route_repair(qr, kr, g: Geom, p: float, k: int, counts, idx, head_work, worklist, workspace,
+                     topp_mask=None, topk_idx=None, stream=None):
+    """fva_route followed by fva_repair in one persistent kernel plus the LPT launch;
+    the Top-p mask and Top-k ids are written only when their tensors are given."""
+    shp = (g.B, g.H, g.N, g.d)
+    _need(qr, torch.bfloat16, shp, "qr")
+    _need(kr, torch.bfloat16, shp, "kr")
+    if topp_mask is not None:
+        _need(topp_mask, torch.uint8, (g.B, g.H, g.Nb, g.Nb), "topp_mask")
+    if topk_idx is not None:
+        _need(topk_idx, torch.int32, (g.B, g.H, g.Nb, min(k, g.Nb)), "topk_idx")
+    _need(counts, torch.int32, (g.B, g.H, g.Nb), "counts")
+    _need(idx, torch.int32, (g.B, g.H, g.Nb, g.Nb), "idx")
+    _need(head_work, torch.int64, (g.B, g.H), "head_work")
+    _need(worklist, torch.int32, (g.B * g.H * g.Nb,), "worklist")
+    _check(lib.fva_route_repair(_ptr(qr), _ptr(kr), g.c(), float(p), int(k), _ptr(topp_mask), _ptr(topk_idx),
+                                _ptr(counts), _ptr(idx), _ptr(head_work), _ptr(worklist), _ptr(workspace),
+                                workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
 def fva_repair_workspace_size(g: Geom) -> int:
     return int(lib.fva_repair_workspace_size(g.c()))
 
@@ -252,12 +273,15 @@ class SparseAttention:
     reorder(Q, K, V) -> route -> repair -> block-sparse attention -> inverse reorder.
 
     Buffers are allocated once through PyTorch for a geometry; `__call__` only
-    enqueues library kernels on the current (or given) stream.
+    enqueues library kernels on the current (or given) stream.  With fused=True
+    (default) routing and repair run as fva_route_repair and the Top-p mask / Top-k
+    ids are not materialised; fused=False runs fva_route then fva_repair.
     """
 
     def __init__(self, g: Geom, p: float, k: int, device="cuda", use_lpt: bool = True,
-                 softmax_scale: float = 0.0):
+                 softmax_scale: float = 0.0, fused: bool = True):
         self.g, self.p, self.k, self.use_lpt, self.scale = g, p, k, use_lpt, softmax_scale
+        self.fused = fused
         dev = torch.device(device)
         shp = (g.B, g.H, g.N, g.d)
         self.qr, self.kr, self.vr, self.outr = (torch.empty(shp, dtype=torch.bfloat16, device=dev) for _ in range(4))
@@ -272,6 +296,10 @@ class SparseAttention:
 
     def routing(self, stream=None) -> None:
         g = self.g
+        if self.fused:
+            fva_route_repair(self.qr, self.kr, g, self.p, self.k, self.rep.counts, self.rep.idx, self.rep.head_work,
+                             self.rep.worklist, self.ws, stream=stream)
+            return
         fva_route(self.qr, self.kr, g, self.p, self.k, self.route.topp_mask, self.route.topk_idx, self.ws,
                   stream=stream)
         fva_repair(self.route.topp_mask, self.route.topk_idx, g, self.k, self.rep.counts, self.rep.idx,

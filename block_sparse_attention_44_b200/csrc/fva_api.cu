@@ -82,7 +82,7 @@ int finish(cudaError_t e, int launches, const char* where) {
 
 extern "C" {
 
-int32_t fva_version(void) { return 100; }
+int32_t fva_version(void) { return 101; }
 
 const char* fva_last_error(void) { return g_err; }
 
@@ -129,9 +129,35 @@ int fva_route(const void* qr, const void* kr, fva_geom g, double p, int32_t k, u
     return fail(FVA_ERR_INVALID_ARG, "workspace too small: %zu bytes given, %zu needed", workspace_bytes, need);
   const int kk = k < D.Nb ? k : D.Nb;
   int launches = 0;
-  cudaError_t e = fva::launch_route(qr, kr, D, p, kk, topp_mask, topk_idx, logits_out, workspace,
+  cudaError_t e = fva::launch_route(qr, kr, D, p, kk, topp_mask, topk_idx, logits_out, nullptr, nullptr, workspace,
                                     static_cast<cudaStream_t>(stream), &launches);
   return finish(e, launches, "fva_route");
+}
+
+int fva_route_repair(const void* qr, const void* kr, fva_geom g, double p, int32_t k, uint8_t* topp_mask,
+                     int32_t* topk_idx, int32_t* counts, int32_t* idx, int64_t* head_work, int32_t* worklist,
+                     void* workspace, size_t workspace_bytes, void* stream) {
+  fva::Dims D;
+  int rc = check_geom(g, D, false);
+  if (rc) return rc;
+  if (!qr || !kr || !counts || !idx || !head_work || !worklist || !workspace)
+    return fail(FVA_ERR_INVALID_ARG, "null pointer");
+  if (!(p > 0.0) || !(p <= 1.0)) return fail(FVA_ERR_INVALID_ARG, "p must satisfy 0 < p <= 1 (got %g)", p);
+  if (k < 1) return fail(FVA_ERR_INVALID_ARG, "k must be >= 1 (got %d)", k);
+  if (D.Nb > fva::kMaxNb) return fail(FVA_ERR_UNSUPPORTED, "Nb = %d blocks exceeds %d", D.Nb, fva::kMaxNb);
+  if (!aligned16(qr) || !aligned16(kr)) return fail(FVA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(FVA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  const size_t need = fva::route_workspace_bytes(D);
+  if (workspace_bytes < need)
+    return fail(FVA_ERR_INVALID_ARG, "workspace too small: %zu bytes given, %zu needed", workspace_bytes, need);
+  const int kk = k < D.Nb ? k : D.Nb;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int launches = 0;
+  cudaError_t e = fva::launch_route(qr, kr, D, p, kk, topp_mask, topk_idx, nullptr, counts, idx, workspace, s,
+                                    &launches);
+  if (e == cudaSuccess) e = fva::launch_lpt(counts, D, head_work, worklist, s, &launches);
+  return finish(e, launches, "fva_route_repair");
 }
 
 size_t fva_repair_workspace_size(fva_geom g) {
@@ -257,7 +283,7 @@ extern "C" int fva_route_static(const void* qr, const void* kr, fva_geom g, doub
   if (!scratch) return fail(FVA_ERR_CUDA, "fva_route_static: cannot resolve the static scratch address");
   const int kk = k < D.Nb ? k : D.Nb;
   int launches = 0;
-  cudaError_t e = fva::launch_route(qr, kr, D, p, kk, topp_mask, topk_idx, logits_out, scratch,
+  cudaError_t e = fva::launch_route(qr, kr, D, p, kk, topp_mask, topk_idx, logits_out, nullptr, nullptr, scratch,
                                     static_cast<cudaStream_t>(stream), &launches);
   return finish(e, launches, "fva_route_static");
 }

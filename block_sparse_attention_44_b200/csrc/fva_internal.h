@@ -21,15 +21,22 @@ constexpr int kMaxNb = 2048;
 cudaError_t launch_reorder(const void* src, void* dst, const fva_geom& g, const Dims& D, bool inverse,
                            cudaStream_t s, int* launches);
 
-// Routing: block means (float64), float64 logits, then the Top-p / Top-k selection.
+// Routing: block means (float64), float64 logits, Top-p / Top-k selection; with
+// counts != nullptr also the repaired, compacted per-row lists (idx, counts).
+// topp_mask, topk_idx and logits_out may each be null (not written).
 cudaError_t launch_route(const void* qr, const void* kr, const Dims& D, double p, int kk, uint8_t* topp_mask,
-                         int32_t* topk_idx, double* logits_out, void* ws, cudaStream_t s, int* launches);
+                         int32_t* topk_idx, double* logits_out, int32_t* counts, int32_t* idx, void* ws,
+                         cudaStream_t s, int* launches);
 size_t route_workspace_bytes(const Dims& D);
 
 // Repair + compaction + per-head work + LPT work list.
 cudaError_t launch_repair(const uint8_t* topp_mask, const int32_t* topk_idx, const Dims& D, int kk, int32_t* counts,
                           int32_t* idx, int64_t* head_work, int32_t* worklist, int* dev_err, cudaStream_t s,
                           int* launches);
+
+// Per-head work W_h and the LPT work list from the per-row counts.
+cudaError_t launch_lpt(const int32_t* counts, const Dims& D, int64_t* head_work, int32_t* worklist, cudaStream_t s,
+                       int* launches);
 
 // Block-sparse attention (tcgen05).
 cudaError_t launch_attention(const void* qr, const void* kr, const void* vr, const int32_t* counts, const int32_t* idx,

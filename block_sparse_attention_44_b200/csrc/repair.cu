@@ -56,14 +56,18 @@ __global__ void __launch_bounds__(kCompactWarps * 32) compact_kernel(const uint8
 }
 
 constexpr int kLptWarps = 16;
+constexpr int kLptBatch = 8;   // counts loaded per lane before they are used
 
+// One CTA.  Items are split into kLptWarps contiguous chunks; warp w histograms its
+// chunk, so a stable scatter only needs, per count value, the number of items in
+// earlier chunks and the running position inside the warp's own chunk.
 __global__ void __launch_bounds__(kLptWarps * 32) lpt_kernel(const int32_t* __restrict__ counts, long long BH, int Nb,
                                                              int64_t* __restrict__ head_work,
                                                              int32_t* __restrict__ worklist) {
   extern __shared__ unsigned lpt_smem[];
-  const int nb1 = Nb + 1;                       // counts are in [1, Nb]
+  const int nb1 = Nb + 1;                       // counts are in [0, Nb]
   unsigned* hist = lpt_smem;                    // [kLptWarps][nb1], later the per-warp cursors
-  unsigned* start = lpt_smem + kLptWarps * nb1; // [nb1]: first position of each count value
+  unsigned* start = lpt_smem + kLptWarps * nb1; // [nb1]: items with a larger count (descending order)
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x & 31;
   const long long n = BH * Nb;
@@ -73,25 +77,50 @@ __global__ void __launch_bounds__(kLptWarps * 32) lpt_kernel(const int32_t* __re
 
   for (int e = threadIdx.x; e < kLptWarps * nb1; e += blockDim.x) hist[e] = 0;
   __syncthreads();
-  for (long long u = lo + lane; u < hi; u += 32) atomicAdd(&hist[warp * nb1 + counts[u]], 1u);
+  for (long long base = lo; base < hi; base += 32 * kLptBatch) {
+    int c[kLptBatch];
+#pragma unroll
+    for (int t = 0; t < kLptBatch; ++t) {
+      const long long u = base + lane + 32 * t;
+      c[t] = u < hi ? __ldg(counts + u) : -1;
+    }
+#pragma unroll
+    for (int t = 0; t < kLptBatch; ++t)
+      if (c[t] >= 0) atomicAdd(&hist[warp * nb1 + c[t]], 1u);
+  }
   // realised per-head workload
   for (long long bh = warp; bh < BH; bh += kLptWarps) {
     long long s = 0;
-    for (int i = lane; i < Nb; i += 32) s += counts[bh * Nb + i];
+    for (int i0 = 0; i0 < Nb; i0 += 32 * kLptBatch) {
+      int c[kLptBatch];
+#pragma unroll
+      for (int t = 0; t < kLptBatch; ++t) {
+        const int i = i0 + lane + 32 * t;
+        c[t] = i < Nb ? __ldg(counts + bh * Nb + i) : 0;
+      }
+#pragma unroll
+      for (int t = 0; t < kLptBatch; ++t) s += c[t];
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
     if (lane == 0) head_work[bh] = s;
   }
   __syncthreads();
-  // start[c] = number of items with a larger count (descending order)
+  // per count value: total over the chunks (kept in start[] for now)
+  for (int v = threadIdx.x; v < nb1; v += blockDim.x) {
+    unsigned t = 0;
+#pragma unroll
+    for (int w = 0; w < kLptWarps; ++w) t += hist[w * nb1 + v];
+    start[v] = t;
+  }
+  __syncthreads();
+  // exclusive scan over count values from high to low (warp 0; lane l owns a run)
   if (warp == 0) {
     const int per = (nb1 + 31) / 32;
-    // lane l owns count values c in (Nb - l*per - per, Nb - l*per], scanned high to low
     unsigned tot = 0;
     for (int q = 0; q < per; ++q) {
-      const int c = Nb - lane * per - q;
-      if (c >= 0)
-        for (int w = 0; w < kLptWarps; ++w) tot += hist[w * nb1 + c];
+      const int v = Nb - lane * per - q;
+      if (v >= 0) tot += start[v];
     }
     unsigned incl = tot;
 #pragma unroll
@@ -101,41 +130,61 @@ __global__ void __launch_bounds__(kLptWarps * 32) lpt_kernel(const int32_t* __re
     }
     unsigned run = incl - tot;
     for (int q = 0; q < per; ++q) {
-      const int c = Nb - lane * per - q;
-      if (c >= 0) {
-        start[c] = run;
-        for (int w = 0; w < kLptWarps; ++w) run += hist[w * nb1 + c];
+      const int v = Nb - lane * per - q;
+      if (v >= 0) {
+        const unsigned t = start[v];
+        start[v] = run;
+        run += t;
       }
     }
   }
   __syncthreads();
-  // per-warp cursors: warp w's items of count c follow those of warps < w
-  for (int c = threadIdx.x; c < nb1; c += blockDim.x) {
-    unsigned run = start[c];
+  // per-warp cursors: warp w's items of count v follow those of warps < w
+  for (int v = threadIdx.x; v < nb1; v += blockDim.x) {
+    unsigned run = start[v];
+#pragma unroll
     for (int w = 0; w < kLptWarps; ++w) {
-      const unsigned t = hist[w * nb1 + c];
-      hist[w * nb1 + c] = run;
+      const unsigned t = hist[w * nb1 + v];
+      hist[w * nb1 + v] = run;
       run += t;
     }
   }
   __syncthreads();
-  // stable scatter, 32 items at a time, in item order within each warp's chunk
-  for (long long b0 = lo; b0 < hi; b0 += 32) {
-    const long long u = b0 + lane;
-    const bool valid = u < hi;
-    const int c = valid ? counts[u] : -1;
-    const unsigned peers = __match_any_sync(0xffffffffu, c);
-    const int rank = __popc(peers & ((1u << lane) - 1u));
-    const int leader = __ffs(peers) - 1;
-    const unsigned basepos = valid ? hist[warp * nb1 + c] : 0u;
-    __syncwarp();
-    if (valid && lane == leader) hist[warp * nb1 + c] = basepos + __popc(peers);
-    __syncwarp();
-    if (valid) worklist[basepos + rank] = static_cast<int32_t>(u);
+  // stable scatter in item order within each warp's chunk, 32 items per step
+  for (long long base = lo; base < hi; base += 32 * kLptBatch) {
+    int c[kLptBatch];
+#pragma unroll
+    for (int t = 0; t < kLptBatch; ++t) {
+      const long long u = base + lane + 32 * t;
+      c[t] = u < hi ? __ldg(counts + u) : -1;
+    }
+#pragma unroll
+    for (int t = 0; t < kLptBatch; ++t) {
+      const long long u = base + lane + 32 * t;
+      const bool valid = c[t] >= 0;
+      const unsigned peers = __match_any_sync(0xffffffffu, c[t]);
+      const int rank = __popc(peers & ((1u << lane) - 1u));
+      const int leader = __ffs(peers) - 1;
+      const unsigned basepos = valid ? hist[warp * nb1 + c[t]] : 0u;
+      __syncwarp();
+      if (valid && lane == leader) hist[warp * nb1 + c[t]] = basepos + __popc(peers);
+      __syncwarp();
+      if (valid) worklist[basepos + rank] = static_cast<int32_t>(u);
+    }
   }
 }
 
 }  // namespace
+
+cudaError_t launch_lpt(const int32_t* counts, const Dims& D, int64_t* head_work, int32_t* worklist, cudaStream_t s,
+                       int* launches) {
+  const size_t lsmem = (static_cast<size_t>(kLptWarps) + 1) * (D.Nb + 1) * sizeof(unsigned);
+  cudaError_t e = cudaFuncSetAttribute(lpt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(lsmem));
+  if (e != cudaSuccess) return e;
+  lpt_kernel<<<1, kLptWarps * 32, lsmem, s>>>(counts, D.BH(), D.Nb, head_work, worklist);
+  ++*launches;
+  return cudaGetLastError();
+}
 
 cudaError_t launch_repair(const uint8_t* topp_mask, const int32_t* topk_idx, const Dims& D, int kk, int32_t* counts,
                           int32_t* idx, int64_t* head_work, int32_t* worklist, int* dev_err, cudaStream_t s,
@@ -145,12 +194,9 @@ cudaError_t launch_repair(const uint8_t* topp_mask, const int32_t* topk_idx, con
   compact_kernel<<<cgrid, kCompactWarps * 32, csmem, s>>>(topp_mask, topk_idx, D.rows(), D.Nb, kk, counts, idx,
                                                           dev_err);
   ++*launches;
-  const size_t lsmem = (static_cast<size_t>(kLptWarps) + 1) * (D.Nb + 1) * sizeof(unsigned);
-  cudaError_t e = cudaFuncSetAttribute(lpt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(lsmem));
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  lpt_kernel<<<1, kLptWarps * 32, lsmem, s>>>(counts, D.BH(), D.Nb, head_work, worklist);
-  ++*launches;
-  return cudaGetLastError();
+  return launch_lpt(counts, D, head_work, worklist, s, launches);
 }
 
 }  // namespace fva

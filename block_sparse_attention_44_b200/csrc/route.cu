@@ -1,19 +1,35 @@
-// Routing frontend: pooled Q/K block scores, Top-p CDF cut, Top-k floor
+// Routing frontend: pooled Q/K block scores, Top-p CDF cut, Top-k floor, and
+// (optionally) the per-row repair and compaction of the kept set
 // ("FVAttn: Adaptive Sparse Attention with Runtime Load Balancing for Video
-// Generation", §2 background on dynamic block-sparse routing and §3.1 overview).
+// Generation", §2 background on dynamic block-sparse routing and §3.1 overview;
+// abstract: the mask is repaired at run time).
 //
-// Three kernels, all float64 so the kept sets agree with an exact computation
-// except at genuine ties:
-//   pool_kernel    — one CTA per (b, h, block) of Q and of K: mean of S bf16 rows.
-//                    HBM-bound, reads every Q/K byte once (S*d*2 bytes per CTA).
-//   logits_kernel  — 64x64-tiled float64 GEMM per (b, h) on the FP64 tensor path:
-//                    L = Qbar Kbar^T / sqrt(d).
-//   select_kernel  — one warp per (b, h, i) row: softmax in float64, masses in 2^-62
-//                    fixed point; the row's Top-p boundary by a 16-step bisection
-//                    over a 1/256-logit bucket index, resolved inside the boundary
-//                    bucket by the exact 64-bit logit key (no sort; integer warp
-//                    sums keep it exact and deterministic); the Top-k floor by
-//                    repeated warp argmax.
+// Two kernels:
+//   pool_kernel   — one CTA per (b, h, block) of Q and of K: the float64 mean of its S
+//                   bf16 rows.  HBM-bound: every Q/K byte is read once here.
+//   select_kernel — one CTA per R query blocks (rows i) of one (b, h): their float64
+//                   logits L_ij = Qbar_i . Kbar_j / sqrt(d) against every key block on
+//                   the FP64 tensor path (mma.sync m8n8k4), then one warp per row:
+//                   softmax, Top-p boundary, Top-k floor, outputs (mask, floor ids,
+//                   logits, compacted kept list).
+// The heads are split into chunks: chunk c is pooled on the caller's stream while a
+// second stream scores and selects chunk c - 1, so selection runs under the memory
+// stream instead of after it.  The two streams meet through events only.
+//
+// Selection arithmetic (deterministic, exact integer sums):
+//   - softmax weights e_j = exp(L_ij - max_j L_ij) in float64, then the mass
+//     m_j = floor(e_j / z * 2^31) (z = sum_j e_j) as an unsigned integer;
+//   - the Top-p boundary is the first position, in the ranking (logit descending,
+//     block id ascending), where the running sum of m reaches ceil(p * 2^31): found
+//     by a 14-step bisection over the bucket index q_j = floor((max L - L_ij) * 256)
+//     (buckets 1/256 logit wide rank like the logits; warp sums by redux.sync), then
+//     inside the boundary bucket by the exact float64 logits;
+//   - the Top-k floor by repeated warp argmax over (logit, -block id).
+// Every mass carries a relative error below 2e-7 and is truncated by less than 2^-31,
+// so the running sum at any cut is within 1.2e-6 of the exact cumulative softmax
+// mass: a kept set can differ from the exact one only where the cumulative mass at
+// the cut lies within that distance of p.
+#include <limits.h>
 #include <math.h>
 
 #include "fva_common.cuh"
@@ -22,9 +38,29 @@
 namespace fva {
 namespace {
 
-// ------------------------------------------------------------------ pooling -------
+constexpr int kRouteThreads = 256;
+constexpr int kRouteWarps = kRouteThreads / 32;
 constexpr int kPoolThreads = 256;
+constexpr int kMaxChunks = 4;           // head chunks overlapped across the two streams
+constexpr unsigned kQCap = 45u * 256u;  // bucket of blocks whose weight e^(L - max) < e^-45 (mass 0)
+constexpr unsigned kQPad = 0xFFFFu;     // bucket of the padding columns past Nb
+constexpr unsigned kFull = 0xffffffffu;
+constexpr int kTopkArgmaxMax = 16;      // floors up to this size use repeated warp argmax
 
+struct RouteArgs {
+  const double* qbar;
+  const double* kbar;
+  uint8_t* topp_mask;   // nullable
+  int32_t* topk_idx;    // nullable
+  double* logits_out;   // nullable
+  int32_t* counts;      // nullable (no compaction when null)
+  int32_t* idx;
+  int Nb, kk;
+  unsigned target;      // ceil(p * 2^31)
+  int keep_all_p;       // p >= 1
+};
+
+// ------------------------------------------------------------------ helpers -------
 __device__ __forceinline__ void bf16x8_to_f64_add(const uint4& v, double (&acc)[8]) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -34,21 +70,55 @@ __device__ __forceinline__ void bf16x8_to_f64_add(const uint4& v, double (&acc)[
   }
 }
 
-// grid.x = 2 * rows: blocks of Q first, then blocks of K.  Means are written to
-// qbar[row] and kbar[row] ([B*H*Nb, D] float64).
+__device__ __forceinline__ double warp_max_f64(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmax(v, __shfl_xor_sync(kFull, v, o));
+  return v;
+}
+__device__ __forceinline__ double warp_sum_f64(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+  return v;
+}
+
+// (L, t) ranks before (L2, t2): logit descending, block id ascending.
+__device__ __forceinline__ bool ranks_before(double L, int t, double L2, int t2) {
+  return L > L2 || (L == L2 && t < t2);
+}
+
+// Warp argmax of (L, t) in ranking order, carrying a payload word.
+__device__ __forceinline__ void warp_argmax(double& L, int& t, unsigned& w) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const double oL = __shfl_xor_sync(kFull, L, o);
+    const int ot = __shfl_xor_sync(kFull, t, o);
+    const unsigned ow = __shfl_xor_sync(kFull, w, o);
+    if (ranks_before(oL, ot, L, t)) {
+      L = oL;
+      t = ot;
+      w = ow;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ pooling -------
+// grid.x = 2 * nrows: blocks row0 .. row0 + nrows - 1 of Q, then the same of K, where
+// block (b*H + h)*Nb + i holds rows [i*S, (i+1)*S) of (b, h).  Thread (rg, col) sums
+// the 16-byte column chunk col over rows rg, rg + RG, ...; the row groups combine in
+// shared memory.  Means go to qbar[block] and kbar[block] ([B*H*Nb, D] float64).
 template <int D>
 __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const uint4* __restrict__ qr, const uint4* __restrict__ kr,
                                                             double* __restrict__ qbar, double* __restrict__ kbar,
-                                                            long long rows, int S) {
+                                                            long long row0, long long nrows, int S) {
   constexpr int CPR = D / 8;                 // 16-byte chunks per row
   constexpr int RG = kPoolThreads / CPR;     // row groups
   __shared__ double part[RG][D];
-  const bool is_k = blockIdx.x >= rows;
-  const long long blk = is_k ? blockIdx.x - rows : blockIdx.x;   // (b*H + h)*Nb + i
+  const bool is_k = blockIdx.x >= nrows;
+  const long long blk = row0 + (is_k ? blockIdx.x - nrows : blockIdx.x);
   const int col = threadIdx.x % CPR;
   const int rg = threadIdx.x / CPR;
   double acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-  const uint4* p = (is_k ? kr : qr) + blk * S * CPR;                // rows of a block are contiguous
+  const uint4* p = (is_k ? kr : qr) + blk * S * CPR;
 #pragma unroll 8
   for (int r = rg; r < S; r += RG) bf16x8_to_f64_add(__ldg(p + r * CPR + col), acc);
 #pragma unroll
@@ -63,357 +133,391 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const uint4* __restr
   }
 }
 
-// ------------------------------------------------------------------ logits --------
-constexpr int kLT = 64;       // output tile (rows and columns) per CTA
-constexpr int kLK = 32;       // reduction chunk staged in shared memory
-constexpr int kLogitThreads = 128;
-
-// L[bh, i, j] = sum_c Qbar[bh, i, c] * Kbar[bh, j, c] / sqrt(D)   (float64)
-// FP64 tensor-core products (mma.sync m8n8k4 f64, exact float64 fused multiply-add
-// per step): each of the four warps owns a 32 x 32 quarter of the 64 x 64 tile as
-// 4 x 4 fragments of 8 x 8; A = Qbar rows, B = Kbar rows (i.e. Kbar^T column-major).
-template <int D>
-__global__ void __launch_bounds__(kLogitThreads) logits_kernel(const double* __restrict__ qbar,
-                                                               const double* __restrict__ kbar,
-                                                               double* __restrict__ L, double* __restrict__ L2,
-                                                               int Nb) {
-  constexpr int LD = kLK + 1;                      // padded row stride (doubles)
-  __shared__ double Qs[kLT][LD];
-  __shared__ double Ks[kLT][LD];
-  const long long bh = blockIdx.z;
-  const int i0 = blockIdx.y * kLT;
-  const int j0 = blockIdx.x * kLT;
-  const int warp = threadIdx.x / 32;
-  const int lane = threadIdx.x & 31;
-  const int gid = lane >> 2, tid = lane & 3;       // mma fragment coordinates
-  const int wi = (warp >> 1) * 32, wj = (warp & 1) * 32;
-  const double* qb = qbar + bh * Nb * D;
-  const double* kb = kbar + bh * Nb * D;
-  double acc[4][4][2];
-#pragma unroll
-  for (int a = 0; a < 4; ++a)
-#pragma unroll
-    for (int c = 0; c < 4; ++c) acc[a][c][0] = acc[a][c][1] = 0.0;
-  for (int c0 = 0; c0 < D; c0 += kLK) {
-    for (int e = threadIdx.x; e < kLT * kLK; e += kLogitThreads) {
-      const int r = e / kLK, c = e - r * kLK;
-      const int gi = i0 + r, gj = j0 + r;
-      Qs[r][c] = gi < Nb ? qb[static_cast<long long>(gi) * D + c0 + c] : 0.0;
-      Ks[r][c] = gj < Nb ? kb[static_cast<long long>(gj) * D + c0 + c] : 0.0;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int k = 0; k < kLK; k += 4) {
-      double a[4], bb[4];
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        a[t] = Qs[wi + 8 * t + gid][k + tid];
-        bb[t] = Ks[wj + 8 * t + gid][k + tid];
-      }
-#pragma unroll
-      for (int ti = 0; ti < 4; ++ti)
-#pragma unroll
-        for (int tj = 0; tj < 4; ++tj)
-          asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
-                       : "+d"(acc[ti][tj][0]), "+d"(acc[ti][tj][1])
-                       : "d"(a[ti]), "d"(bb[tj]));
-    }
-    __syncthreads();
-  }
-  const double rs = sqrt(static_cast<double>(D));
-#pragma unroll
-  for (int ti = 0; ti < 4; ++ti) {
-    const int i = i0 + wi + 8 * ti + gid;
-    if (i >= Nb) continue;
-#pragma unroll
-    for (int tj = 0; tj < 4; ++tj)
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int j = j0 + wj + 8 * tj + 2 * tid + e;
-        if (j >= Nb) continue;
-        const double val = acc[ti][tj][e] / rs;
-        const long long o = (bh * Nb + i) * static_cast<long long>(Nb) + j;
-        L[o] = val;
-        if (L2) L2[o] = val;
-      }
-  }
-}
-
 // ------------------------------------------------------------------ selection -----
-constexpr int kSelWarps = 4;
-constexpr int kTopkArgmaxMax = 16;   // floors up to this size use repeated warp argmax
-typedef unsigned long long u64;
-
-// Order-preserving map of a float64 logit to an unsigned key (larger logit -> larger key).
-__device__ __forceinline__ u64 order_key(double L) {
-  if (L == 0.0) L = 0.0;  // -0 and +0 rank equal
-  const u64 u = static_cast<u64>(__double_as_longlong(L));
-  return (u & 0x8000000000000000ull) ? ~u : (u | 0x8000000000000000ull);
-}
-
-__device__ __forceinline__ u64 warp_sum_u64(u64 v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
-
-// Boundary of the ranking (key descending, block id ascending) where the running
-// weight first reaches `target` (weight = fixed-point mass, or 1 per block when
-// !by_mass).  Requires 0 < target <= total weight.
-//   1. Bisection over q = min(65535, floor((Lmax - L) * 256)), which ranks like the
-//      logit in steps of 1/256: the boundary bucket q* is the smallest q whose
-//      bucket-inclusive weight reaches the target (16 integer-sum steps).
-//   2. Inside bucket q* (blocks within 1/256 of each other) the exact order is taken
-//      from the 64-bit keys: repeated warp argmax until the weight reaches the target.
-// All sums are warp reductions of integers: exact and deterministic.  Outputs the
-// boundary's key and block id, and its 1-based rank.
-__device__ void warp_select(const u64* key, const u64* mass, const unsigned* qk, int Nb, u64 target, bool by_mass,
-                            u64& bkey, int& bj, int& rank) {
-  const int lane = threadIdx.x & 31;
-  unsigned lo = 0, hi = 65535;
+// Smallest q in [lo, hi] whose bucket-inclusive weight sum reaches T (weight = mass,
+// or 1 per block when !BY_MASS).  Requires the weight of bucket hi to reach T.
+template <int PL, bool BY_MASS>
+__device__ __forceinline__ unsigned bisect(const unsigned (&q)[PL], const unsigned (&m)[PL], unsigned lo, unsigned hi,
+                                           unsigned T) {
   while (lo < hi) {
     const unsigned mid = (lo + hi) >> 1;
-    u64 w = 0;
-    for (int t = lane; t < Nb; t += 32)
-      if (qk[t] <= mid) w += by_mass ? mass[t] : 1ull;
-    w = warp_sum_u64(w);
-    if (w >= target)
+    unsigned w = 0;
+#pragma unroll
+    for (int s = 0; s < PL; ++s)
+      if (q[s] <= mid) w += BY_MASS ? m[s] : 1u;
+    w = __reduce_add_sync(kFull, w);
+    if (w >= T)
       hi = mid;
     else
       lo = mid + 1;
   }
-  const unsigned qs = lo;
-  u64 above_w = 0;
-  unsigned above_n = 0;
-  for (int t = lane; t < Nb; t += 32)
-    if (qk[t] < qs) {
-      above_w += by_mass ? mass[t] : 1ull;
-      ++above_n;
-    }
-  above_w = warp_sum_u64(above_w);
+  return lo;
+}
+
+// Walks bucket qs in ranking order from weight `acc` (the weight of every better
+// bucket) until the running weight reaches T; returns that block's (logit, id).
+template <int PL, bool BY_MASS>
+__device__ __forceinline__ void walk_bucket(const double* Lr, const unsigned (&q)[PL], const unsigned (&m)[PL], unsigned qs,
+                            unsigned acc, unsigned T, double& Lb, int& jb) {
+  const int lane = threadIdx.x & 31;
+  double Lp = INFINITY;
+  int jp = -1;
+  for (int guard = 0; guard < 32 * PL; ++guard) {
+    double bL = -INFINITY;
+    int bt = INT_MAX;
+    unsigned bw = 0;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) above_n += __shfl_xor_sync(0xffffffffu, above_n, o);
-  // walk bucket qs in exact order: key descending, block id ascending
-  u64 prev_key = ~0ull;
-  int prev_j = -1;
-  for (int guard = 0; guard < Nb; ++guard) {
-    u64 best = 0;
-    int bjx = 0x7fffffff;
-    for (int t = lane; t < Nb; t += 32) {
-      if (qk[t] != qs) continue;
-      const u64 kv = key[t];
-      // strictly after (prev_key, prev_j) in the ranking
-      const bool after = kv < prev_key || (kv == prev_key && t > prev_j);
-      if (after && (kv > best || (kv == best && t < bjx))) {
-        best = kv;
-        bjx = t;
+    for (int s = 0; s < PL; ++s) {
+      if (q[s] != qs) continue;
+      const int t = lane + 32 * s;
+      const double L = Lr[t];
+      if (ranks_before(Lp, jp, L, t) && ranks_before(L, t, bL, bt)) {
+        bL = L;
+        bt = t;
+        bw = BY_MASS ? m[s] : 1u;
       }
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const u64 ob = __shfl_xor_sync(0xffffffffu, best, o);
-      const int oj = __shfl_xor_sync(0xffffffffu, bjx, o);
-      if (ob > best || (ob == best && oj < bjx)) {
-        best = ob;
-        bjx = oj;
-      }
-    }
-    if (bjx == 0x7fffffff) break;               // bucket exhausted (cannot happen)
-    above_w += by_mass ? mass[bjx] : 1ull;
-    ++above_n;
-    prev_key = best;
-    prev_j = bjx;
-    if (above_w >= target) {
-      bkey = best;
-      bj = bjx;
-      rank = static_cast<int>(above_n);
+    warp_argmax(bL, bt, bw);
+    if (bt == INT_MAX) break;   // bucket exhausted: cannot happen when the bucket reaches T
+    acc += bw;
+    if (acc >= T) {
+      Lb = bL;
+      jb = bt;
       return;
     }
+    Lp = bL;
+    jp = bt;
   }
-  // unreachable when 0 < target <= total: keep everything
-  bkey = 0;
-  bj = Nb;
-  rank = Nb;
+  Lb = -INFINITY;   // keep everything
+  jb = INT_MAX;
 }
 
-// Per-warp shared memory of select_kernel: keys and masses (8 bytes) and bucket
-// indices (4 bytes) per block, rounded up so every warp's 8-byte arrays stay aligned.
-__host__ __device__ constexpr size_t sel_bytes_per_warp(int Nb) {
-  return ((2 * sizeof(u64) + sizeof(unsigned)) * static_cast<size_t>(Nb) + 15) & ~static_cast<size_t>(15);
-}
-
-__global__ void __launch_bounds__(kSelWarps * 32) select_kernel(const double* __restrict__ L, long long rows, int Nb,
-                                                                double p, int kk, uint8_t* __restrict__ topp_mask,
-                                                                int32_t* __restrict__ topk_idx) {
-  extern __shared__ __align__(16) unsigned char sel_smem[];
-  const int warp = threadIdx.x / 32;
+// Row i of (b, h) = bh; Lr = its logits in shared memory (32*PL entries, -inf past Nb).
+template <int PL>
+__device__ __forceinline__ void select_row(const RouteArgs& a, long long bh, int i, const double* Lr) {
   const int lane = threadIdx.x & 31;
-  const long long row = static_cast<long long>(blockIdx.x) * kSelWarps + warp;
-  if (row >= rows) return;
-  const size_t per_warp = sel_bytes_per_warp(Nb);
-  u64* key = reinterpret_cast<u64*>(sel_smem + per_warp * warp);
-  u64* mass = key + Nb;
-  unsigned* qk = reinterpret_cast<unsigned*>(mass + Nb);
-  const double* Lr = L + row * Nb;
+  const int Nb = a.Nb;
+  const long long row = bh * Nb + i;
 
   double mx = -INFINITY;
-  for (int t = lane; t < Nb; t += 32) mx = fmax(mx, Lr[t]);
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  // blocks more than 45 below the row max carry a probability below e^-45 < 2^-64,
-  // which is exactly zero in the 2^-62 fixed point: their exponential is skipped
+  for (int s = 0; s < PL; ++s) mx = fmax(mx, Lr[lane + 32 * s]);
+  mx = warp_max_f64(mx);
+
+  // weights, bucket indices; e^-45 < 2^-64: those blocks carry mass 0 and go to kQCap
+  unsigned q[PL], m[PL];
   double z = 0.0;
-  for (int t = lane; t < Nb; t += 32) {
-    const double l = Lr[t];
-    key[t] = order_key(l);
-    const double d = l - mx;
-    const double e = d > -45.0 ? exp(d) : 0.0;
-    mass[t] = static_cast<u64>(__double_as_longlong(e));  // raw bits for now
-    const double qd = -d * 256.0;
-    qk[t] = qd < 65535.0 ? static_cast<unsigned>(qd) : 65535u;
+#pragma unroll
+  for (int s = 0; s < PL; ++s) {
+    const int t = lane + 32 * s;
+    const double d = Lr[t] - mx;
+    const bool live = d > -45.0;
+    const double e = live ? exp(d) : 0.0;
     z += e;
+    m[s] = __float_as_uint(__double2float_rn(e));
+    q[s] = live ? static_cast<unsigned>(-d * 256.0) : (t < Nb ? kQCap : kQPad);
   }
+  z = warp_sum_f64(z);
+  const float scale = __double2float_rn(0x1p31 / z);
+  unsigned part = 0;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-  const double to_fixed = 0x1p62 / z;
-  u64 tot = 0;
-  for (int t = lane; t < Nb; t += 32) {
-    const double e = __longlong_as_double(static_cast<long long>(mass[t]));
-    const u64 m = static_cast<u64>(e * to_fixed);
-    mass[t] = m;
-    tot += m;
+  for (int s = 0; s < PL; ++s) {
+    m[s] = __float2uint_rz(__uint_as_float(m[s]) * scale);
+    part += m[s];
   }
-  tot = warp_sum_u64(tot);
-  __syncwarp();
+  const unsigned tot = __reduce_add_sync(kFull, part);
 
-  // Top-p boundary
-  bool keep_all = p >= 1.0;
-  u64 bkey_p = 0;
-  int bj_p = Nb, n_p = Nb;
-  if (!keep_all) {
-    u64 target = static_cast<u64>(p * 0x1p62);
-    if (target == 0) target = 1;
-    if (tot < target) {
-      keep_all = true;
-    } else {
-      warp_select(key, mass, qk, Nb, target, true, bkey_p, bj_p, n_p);
-    }
+  // Top-p boundary (Lp_b, jp_b): the kept set is every block ranking at or before it
+  const bool all_p = a.keep_all_p || tot < a.target;
+  unsigned qp = 0;
+  double Lpb = -INFINITY;
+  int jpb = INT_MAX;
+  if (!all_p) {
+    qp = bisect<PL, true>(q, m, 0u, kQCap - 1u, a.target);
+    unsigned above = 0;
+#pragma unroll
+    for (int s = 0; s < PL; ++s)
+      if (q[s] < qp) above += m[s];
+    above = __reduce_add_sync(kFull, above);
+    walk_bucket<PL, true>(Lr, q, m, qp, above, a.target, Lpb, jpb);
   }
 
-  uint8_t* mrow = topp_mask + row * Nb;
-  for (int t = lane; t < Nb; t += 32) {
-    const u64 kv = key[t];
-    const bool in = keep_all || kv > bkey_p || (kv == bkey_p && t <= bj_p);
-    mrow[t] = in ? 1 : 0;
-  }
-
-  // Top-k floor: the kk highest-ranked blocks (key descending, block id ascending),
-  // by repeated warp argmax for a small floor, by radix select otherwise
-  int32_t* krow = topk_idx + row * kk;
+  // Top-k floor
+  const int kk = a.kk;
+  unsigned long long taken = 0;   // bit s: block lane + 32 s is in the floor (kk <= kTopkArgmaxMax)
+  unsigned qk = 0;
+  double Lkb = -INFINITY;
+  int jkb = INT_MAX;
+  int32_t* krow = a.topk_idx ? a.topk_idx + row * kk : nullptr;
   if (kk <= kTopkArgmaxMax) {
-    unsigned taken = 0, taken_hi = 0;   // bit s: element lane + 32*s already chosen (s < 64 as Nb <= 2048)
-    int chosen[kTopkArgmaxMax];
-    for (int q = 0; q < kk; ++q) {
-      u64 best = 0;
-      int bjx = 0x7fffffff;
-      for (int t = lane, sidx = 0; t < Nb; t += 32, ++sidx) {
-        const bool tk = sidx < 32 ? ((taken >> sidx) & 1u) : ((taken_hi >> (sidx - 32)) & 1u);
-        const u64 kv = key[t];
-        if (!tk && (kv > best || (kv == best && t < bjx))) {
-          best = kv;
-          bjx = t;
-        }
-      }
+    int mine = INT_MAX;   // lane c holds the c-th chosen id
+    for (int c = 0; c < kk; ++c) {
+      double bL = -INFINITY;
+      int bt = INT_MAX;
+      unsigned bs = 0;
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const u64 ob = __shfl_xor_sync(0xffffffffu, best, o);
-        const int oj = __shfl_xor_sync(0xffffffffu, bjx, o);
-        if (ob > best || (ob == best && oj < bjx)) {
-          best = ob;
-          bjx = oj;
+      for (int s = 0; s < PL; ++s) {
+        const int t = lane + 32 * s;
+        if (((taken >> s) & 1ull) || t >= Nb) continue;
+        const double L = Lr[t];
+        if (ranks_before(L, t, bL, bt)) {
+          bL = L;
+          bt = t;
+          bs = static_cast<unsigned>(s);
         }
       }
-      chosen[q] = bjx;
-      if ((bjx & 31) == lane) {
-        const int sidx = bjx >> 5;
-        if (sidx < 32)
-          taken |= 1u << sidx;
-        else
-          taken_hi |= 1u << (sidx - 32);
-      }
+      warp_argmax(bL, bt, bs);
+      if ((bt & 31) == lane) taken |= 1ull << bs;
+      if (lane == c) mine = bt;
     }
-    // write in ascending block id (chosen[] is identical in every lane)
-    if (lane == 0) {
-      for (int a = 1; a < kk; ++a) {
-        const int v = chosen[a];
-        int b2 = a - 1;
-        while (b2 >= 0 && chosen[b2] > v) {
-          chosen[b2 + 1] = chosen[b2];
-          --b2;
-        }
-        chosen[b2 + 1] = v;
-      }
-      for (int a = 0; a < kk; ++a) krow[a] = chosen[a];
+    if (krow) {   // ascending block id: lane c writes its id at its rank
+      int rank = 0;
+      for (int c = 0; c < kk; ++c) rank += __shfl_sync(kFull, mine, c) < mine ? 1 : 0;
+      if (lane < kk) krow[rank] = mine;
     }
   } else {
-    u64 bkey_k;
-    int bj_k, n_k;
-    warp_select(key, mass, qk, Nb, static_cast<u64>(kk), false, bkey_k, bj_k, n_k);
-    int pos = 0;
-    for (int base = 0; base < Nb; base += 32) {
-      const int t = base + lane;
-      bool in = false;
-      if (t < Nb) {
-        const u64 kv = key[t];
-        in = kv > bkey_k || (kv == bkey_k && t <= bj_k);
-      }
-      const unsigned bal = __ballot_sync(0xffffffffu, in);
-      if (in) krow[pos + __popc(bal & ((1u << lane) - 1u))] = t;
+    qk = bisect<PL, false>(q, m, 0u, kQCap, static_cast<unsigned>(kk));
+    unsigned above = 0;
+#pragma unroll
+    for (int s = 0; s < PL; ++s)
+      if (q[s] < qk) ++above;
+    above = __reduce_add_sync(kFull, above);
+    walk_bucket<PL, false>(Lr, q, m, qk, above, static_cast<unsigned>(kk), Lkb, jkb);
+  }
+
+  // outputs: Top-p mask, floor ids (large floors), logits, compacted kept list
+  uint8_t* mrow = a.topp_mask ? a.topp_mask + row * Nb : nullptr;
+  double* lrow = a.logits_out ? a.logits_out + row * Nb : nullptr;
+  int32_t* irow = a.counts ? a.idx + row * Nb : nullptr;
+  const bool big_k = kk > kTopkArgmaxMax;
+  int kpos = 0, pos = 0;
+#pragma unroll
+  for (int s = 0; s < PL; ++s) {
+    if (32 * s >= Nb) break;
+    const int t = lane + 32 * s;
+    const bool valid = t < Nb;
+    const double L = Lr[t];
+    const bool in_p = valid && (all_p || q[s] < qp || (q[s] == qp && !ranks_before(Lpb, jpb, L, t)));
+    const bool in_k = big_k ? valid && (q[s] < qk || (q[s] == qk && !ranks_before(Lkb, jkb, L, t)))
+                            : ((taken >> s) & 1ull) != 0;
+    if (valid && mrow) mrow[t] = in_p ? 1 : 0;
+    if (valid && lrow) lrow[t] = L;
+    if (big_k) {
+      const unsigned bal = __ballot_sync(kFull, in_k);
+      if (in_k && krow) krow[kpos + __popc(bal & ((1u << lane) - 1u))] = t;
+      kpos += __popc(bal);
+    }
+    if (irow) {
+      const bool keep = in_p || in_k || t == i;
+      const unsigned bal = __ballot_sync(kFull, valid && keep);
+      if (valid && keep) irow[pos + __popc(bal & ((1u << lane) - 1u))] = t;
       pos += __popc(bal);
     }
   }
+  if (irow && lane == 0) a.counts[row] = pos;
+}
+
+// R query blocks [i0, i0 + R) of bh: logits into shared memory, then one warp per row.
+template <int D, int PL, int R, int KU>
+__device__ __forceinline__ void select_item(const RouteArgs& a, long long bh, int i0, unsigned char* smem) {
+  constexpr int LDQ = D + 4;             // padded rows (8-byte words)
+  constexpr int LDL = 32 * PL + 2;
+  constexpr int NT = 4 * PL;             // 8-column tiles covering 32 * PL columns
+  double* Qs = reinterpret_cast<double*>(smem);
+  double* Ls = Qs + R * LDQ;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int Nb = a.Nb;
+
+  const double* qb = a.qbar + bh * Nb * D;
+  const double* kb = a.kbar + bh * Nb * D;
+  for (int e = tid; e < R * D; e += kRouteThreads) {
+    const int r = e / D, c = e - r * D;
+    Qs[r * LDQ + c] = i0 + r < Nb ? __ldcg(qb + static_cast<long long>(i0 + r) * D + c) : 0.0;
+  }
+  __syncthreads();
+
+  // L = Qbar Kbar^T / sqrt(D): warp w takes column tiles w, w + 8, w + 16, ... four at
+  // a time, so each A fragment feeds four independent accumulation chains.  Fragment
+  // coordinates of m8n8k4 (row.col): A[gid][tq], B[tq][gid], C[gid][2 tq + e].
+  static_assert(R == 8, "one 8-row MMA tile per item");
+  constexpr int NTW = NT / kRouteWarps;          // column tiles per warp
+  const int gid = lane >> 2, tq = lane & 3;
+  const int ntv = (Nb + 7) / 8;
+  const double rs = sqrt(static_cast<double>(D));
+  const double* qa = Qs + gid * LDQ + tq;
+#pragma unroll 1
+  for (int j0 = 0; j0 < NTW; j0 += 4) {
+    double acc[4][2];
+    const double* kp[4];
+    bool jv[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int nt = warp + kRouteWarps * (j0 + u);
+      const int j = nt * 8 + gid;
+      jv[u] = j0 + u < NTW && nt < ntv && j < Nb;
+      kp[u] = kb + static_cast<long long>(jv[u] ? j : 0) * D + tq;
+      acc[u][0] = acc[u][1] = 0.0;
+    }
+#pragma unroll KU
+    for (int k = 0; k < D; k += 4) {
+      const double av = qa[k];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const double b = jv[u] ? __ldcg(kp[u] + k) : 0.0;
+        asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+                     : "+d"(acc[u][0]), "+d"(acc[u][1])
+                     : "d"(av), "d"(b));
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (j0 + u >= NTW) break;
+      const int nt = warp + kRouteWarps * (j0 + u);
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int c = nt * 8 + 2 * tq + e;
+        Ls[gid * LDL + c] = c < Nb ? acc[u][e] / rs : -INFINITY;
+      }
+    }
+  }
+  __syncthreads();
+
+  for (int r = warp; r < R; r += kRouteWarps)
+    if (i0 + r < Nb) select_row<PL>(a, bh, i0 + r, Ls + r * LDL);
+}
+
+template <int D, int PL, int R>
+constexpr size_t select_smem_bytes() {
+  return (static_cast<size_t>(R) * (D + 4) + static_cast<size_t>(R) * (32 * PL + 2)) * sizeof(double);
+}
+
+// grid = (ceil(Nb / R), heads): CTA (x, y) selects rows [x*R, x*R + R) of (b, h) = bh0 + y.
+// MINB CTAs per SM; KU = unrolled k-steps of the logits loop for that register budget.
+template <int D, int PL, int R, int MINB>
+__global__ void __launch_bounds__(kRouteThreads, MINB) select_kernel(const RouteArgs a, long long bh0) {
+  constexpr int KU = MINB >= 4 ? 2 : (MINB == 3 ? 4 : 8);
+  extern __shared__ __align__(16) unsigned char sel_smem[];
+  select_item<D, PL, R, KU>(a, bh0 + blockIdx.y, static_cast<int>(blockIdx.x) * R, sel_smem);
 }
 
 size_t align_up(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+struct Carve {
+  double* qbar;
+  double* kbar;
+};
+
+Carve carve(const Dims& D, void* ws) {
+  const size_t pooled = align_up(static_cast<size_t>(D.rows()) * D.d * sizeof(double));
+  unsigned char* w = static_cast<unsigned char*>(ws);
+  return Carve{reinterpret_cast<double*>(w), reinterpret_cast<double*>(w + pooled)};
+}
+
+// The second stream and the fork/join events, per host thread and device (a thread
+// never shares them, so concurrent callers on other threads cannot interleave).
+struct SideStream {
+  cudaStream_t stream = nullptr;
+  cudaEvent_t ev[kMaxChunks + 2] = {};
+  bool ready = false;
+};
+
+cudaError_t side_stream(SideStream** out) {
+  thread_local SideStream ctx[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  SideStream& c = ctx[dev];
+  if (!c.ready) {
+    int lo = 0, hi = 0;
+    e = cudaDeviceGetStreamPriorityRange(&lo, &hi);
+    if (e != cudaSuccess) return e;
+    e = cudaStreamCreateWithPriority(&c.stream, cudaStreamNonBlocking, hi);   // selection first when both wait
+    if (e != cudaSuccess) return e;
+    for (auto& ev : c.ev) {
+      e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming);
+      if (e != cudaSuccess) return e;
+    }
+    c.ready = true;
+  }
+  *out = &c;
+  return cudaSuccess;
+}
+
+template <int D, int PL, int R, int MINB>
+cudaError_t launch_select_variant(const RouteArgs& a, long long bh0, long long nbh, cudaStream_t s) {
+  auto kern = select_kernel<D, PL, R, MINB>;
+  constexpr size_t smem = select_smem_bytes<D, PL, R>();
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const dim3 grid(static_cast<unsigned>((a.Nb + R - 1) / R), static_cast<unsigned>(nbh));
+  kern<<<grid, kRouteThreads, smem, s>>>(a, bh0);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_select(const RouteArgs& a, long long bh0, long long nbh, cudaStream_t s) {
+  if (a.Nb <= 256) return launch_select_variant<D, 8, 8, 4>(a, bh0, nbh, s);
+  if (a.Nb <= 640) return launch_select_variant<D, 20, 8, 3>(a, bh0, nbh, s);
+  if (a.Nb <= 1280) return launch_select_variant<D, 40, 8, 2>(a, bh0, nbh, s);
+  return launch_select_variant<D, 64, 8, 1>(a, bh0, nbh, s);
+}
 
 }  // namespace
 
 size_t route_workspace_bytes(const Dims& D) {
   const size_t pooled = static_cast<size_t>(D.rows()) * D.d * sizeof(double);
-  const size_t logits = static_cast<size_t>(D.rows()) * D.Nb * sizeof(double);
-  return 2 * align_up(pooled) + align_up(logits);
+  return 2 * align_up(pooled);
 }
 
 cudaError_t launch_route(const void* qr, const void* kr, const Dims& D, double p, int kk, uint8_t* topp_mask,
-                         int32_t* topk_idx, double* logits_out, void* ws, cudaStream_t s, int* launches) {
-  const size_t pooled = align_up(static_cast<size_t>(D.rows()) * D.d * sizeof(double));
-  unsigned char* w = static_cast<unsigned char*>(ws);
-  double* qbar = reinterpret_cast<double*>(w);
-  double* kbar = reinterpret_cast<double*>(w + pooled);
-  double* L = reinterpret_cast<double*>(w + 2 * pooled);
-  const dim3 pgrid(static_cast<unsigned>(2 * D.rows()));
-  if (D.d == 128)
-    pool_kernel<128><<<pgrid, kPoolThreads, 0, s>>>(static_cast<const uint4*>(qr), static_cast<const uint4*>(kr), qbar,
-                                                    kbar, D.rows(), D.S);
-  else
-    pool_kernel<64><<<pgrid, kPoolThreads, 0, s>>>(static_cast<const uint4*>(qr), static_cast<const uint4*>(kr), qbar,
-                                                   kbar, D.rows(), D.S);
-  ++*launches;
-  const int nt = (D.Nb + kLT - 1) / kLT;
-  const dim3 lgrid(nt, nt, static_cast<unsigned>(D.BH()));
-  if (D.d == 128)
-    logits_kernel<128><<<lgrid, kLogitThreads, 0, s>>>(qbar, kbar, L, logits_out, D.Nb);
-  else
-    logits_kernel<64><<<lgrid, kLogitThreads, 0, s>>>(qbar, kbar, L, logits_out, D.Nb);
-  ++*launches;
-  const size_t smem = kSelWarps * sel_bytes_per_warp(D.Nb);
-  cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+                         int32_t* topk_idx, double* logits_out, int32_t* counts, int32_t* idx, void* ws,
+                         cudaStream_t s, int* launches) {
+  const Carve c = carve(D, ws);
+  RouteArgs a;
+  a.qbar = c.qbar;
+  a.kbar = c.kbar;
+  a.topp_mask = topp_mask;
+  a.topk_idx = topk_idx;
+  a.logits_out = logits_out;
+  a.counts = counts;
+  a.idx = idx;
+  a.Nb = D.Nb;
+  a.kk = kk;
+  a.keep_all_p = p >= 1.0 ? 1 : 0;
+  const double tp = ceil(p * 0x1p31);
+  a.target = a.keep_all_p ? 0u : static_cast<unsigned>(tp < 1.0 ? 1.0 : tp);
+
+  SideStream* side = nullptr;
+  cudaError_t e = side_stream(&side);
   if (e != cudaSuccess) return e;
-  const unsigned sgrid = static_cast<unsigned>((D.rows() + kSelWarps - 1) / kSelWarps);
-  select_kernel<<<sgrid, kSelWarps * 32, smem, s>>>(L, D.rows(), D.Nb, p, kk, topp_mask, topk_idx);
-  ++*launches;
-  return cudaGetLastError();
+  const long long BH = D.BH();
+  const int nchunks = static_cast<int>(BH < kMaxChunks ? BH : kMaxChunks);
+  // fork: the side stream starts after everything already queued on s
+  if ((e = cudaEventRecord(side->ev[0], s)) != cudaSuccess) return e;
+  if ((e = cudaStreamWaitEvent(side->stream, side->ev[0], 0)) != cudaSuccess) return e;
+  for (int ch = 0; ch < nchunks; ++ch) {
+    const long long bh0 = BH * ch / nchunks, bh1 = BH * (ch + 1) / nchunks;
+    const long long row0 = bh0 * D.Nb, nrows = (bh1 - bh0) * D.Nb;
+    const dim3 pgrid(static_cast<unsigned>(2 * nrows));
+    if (D.d == 128)
+      pool_kernel<128><<<pgrid, kPoolThreads, 0, s>>>(static_cast<const uint4*>(qr), static_cast<const uint4*>(kr),
+                                                      c.qbar, c.kbar, row0, nrows, D.S);
+    else
+      pool_kernel<64><<<pgrid, kPoolThreads, 0, s>>>(static_cast<const uint4*>(qr), static_cast<const uint4*>(kr),
+                                                     c.qbar, c.kbar, row0, nrows, D.S);
+    ++*launches;
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = cudaEventRecord(side->ev[ch + 1], s)) != cudaSuccess) return e;
+    if ((e = cudaStreamWaitEvent(side->stream, side->ev[ch + 1], 0)) != cudaSuccess) return e;
+    e = D.d == 128 ? launch_select<128>(a, bh0, bh1 - bh0, side->stream)
+                   : launch_select<64>(a, bh0, bh1 - bh0, side->stream);
+    ++*launches;
+    if (e != cudaSuccess) return e;
+  }
+  // join: later work on s sees every selection
+  if ((e = cudaEventRecord(side->ev[kMaxChunks + 1], side->stream)) != cudaSuccess) return e;
+  return cudaStreamWaitEvent(s, side->ev[kMaxChunks + 1], 0);
 }
 
 }  // namespace fva

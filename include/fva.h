@@ -9,6 +9,7 @@
  *   fva_route            pooled Q/K block scores, Top-p CDF cut, Top-k floor
  *   fva_repair           forced diagonal + floor, compaction into per-row key-block lists,
  *                        per-head realised workload, heavy-first (LPT) work list
+ *   fva_route_repair     the two above, fused
  *   fva_block_sparse_attn  flash-style attention over the kept block pairs
  *   fva_inverse_reorder  back to natural token order
  *
@@ -66,7 +67,7 @@ int fva_reorder(const void* x, void* xr, fva_geom g, void* stream);
  */
 int fva_inverse_reorder(const void* xr, void* x, fva_geom g, void* stream);
 
-/* Workspace bytes fva_route needs for geometry g (pooled Q/K and block logits, float64). */
+/* Workspace bytes fva_route needs for geometry g (pooled Q and K, float64). */
 size_t fva_route_workspace_size(fva_geom g);
 
 /*
@@ -81,8 +82,16 @@ size_t fva_route_workspace_size(fva_geom g);
  *                blocks of each row, in ascending block id.
  *   logits_out : optional float64 [B,H,Nb,Nb] output of Qbar_i.Kbar_j/sqrt(d), or NULL.
  * Arithmetic: per-block means and logits in float64; rows ranked by logit descending,
- * ties to the lower block id; the cumulative mass of the softmax is accumulated in
- * 2^-62 fixed point, so the result is deterministic.  Requires Nb <= 2048.
+ * ties to the lower block id.  Softmax masses are the float64 weights exp(L - max L)
+ * normalised and truncated to 2^-31 fixed point; the running mass is an exact integer
+ * sum, so the result is deterministic and the cumulative mass at any cut is within
+ * 1.2e-6 of the exact one (a kept set differs from the exact rule only where the
+ * cumulative mass at the cut lies that close to p).  Requires Nb <= 2048.
+ * Launches: per head chunk (up to 4) a pooling kernel on `stream` and a selection
+ * kernel on a second stream the library owns (one per host thread and device), so the
+ * selection of a chunk runs while the next chunk is pooled; the second stream starts
+ * after the work already queued on `stream` and `stream` waits for it before the call
+ * returns (events), so everything stays ordered on `stream`, graph capture included.
  */
 int fva_route(const void* qr, const void* kr, fva_geom g, double p, int32_t k,
               uint8_t* topp_mask, int32_t* topk_idx, double* logits_out,
@@ -101,8 +110,9 @@ int fva_route(const void* qr, const void* kr, fva_geom g, double p, int32_t k,
  * FVA_ROUTE_STATIC_SCRATCH_BYTES (64 MiB), reserved on every GPU that loads this
  * library and held until the process exits.
  *   - Geometries whose fva_route_workspace_size() exceeds that size are rejected with
- *     FVA_ERR_UNSUPPORTED and a message; nothing is enqueued.  (The 480p layer,
- *     B=1 H=40 d=128 with 240 blocks, needs about 36 MiB; the 720p layer does not fit.)
+ *     FVA_ERR_UNSUPPORTED and a message; nothing is enqueued.  (The 720p layer,
+ *     B=1 H=40 d=128 with 600 blocks, needs about 47 MiB; with 64-token tiles, 1200
+ *     blocks, it needs about 94 MiB and does not fit.)
  *   - Nothing in the scratch needs to start at zero: each call writes every scratch
  *     byte it later reads.  The array keeps the last call's contents.
  *   - All calls on a device share the one array: calls whose GPU execution overlaps
@@ -114,6 +124,21 @@ int fva_route(const void* qr, const void* kr, fva_geom g, double p, int32_t k,
 #define FVA_ROUTE_STATIC_SCRATCH_BYTES ((size_t)64 << 20)
 int fva_route_static(const void* qr, const void* kr, fva_geom g, double p, int32_t k,
                      uint8_t* topp_mask, int32_t* topk_idx, double* logits_out, void* stream);
+
+/*
+ * fva_route_repair — fva_route followed by fva_repair, fused (same outputs, same
+ * arithmetic; the pages describe the two steps, not their split into calls).
+ * The per-row repair and compaction run inside fva_route's selection kernel (no
+ * mask round trip through memory); one more launch on `stream` builds head_work and
+ * the LPT work list.
+ *   workspace        : fva_route_workspace_size(g) bytes.
+ *   topp_mask, topk_idx : as in fva_route, or NULL when the caller does not need them.
+ *   counts, idx, head_work, worklist : as in fva_repair (required).
+ */
+int fva_route_repair(const void* qr, const void* kr, fva_geom g, double p, int32_t k,
+                     uint8_t* topp_mask, int32_t* topk_idx, int32_t* counts, int32_t* idx,
+                     int64_t* head_work, int32_t* worklist,
+                     void* workspace, size_t workspace_bytes, void* stream);
 
 /* Workspace bytes fva_repair needs (currently 0; kept for ABI stability). */
 size_t fva_repair_workspace_size(fva_geom g);

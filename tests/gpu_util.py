@@ -45,13 +45,34 @@ def run_path(fva, g, q, k, v, p, kfloor, use_lpt=True, want_logits=False):
     hw = torch.empty((g.B, g.H), dtype=torch.int64, device="cuda")
     wl = torch.empty((g.B * g.H * g.Nb,), dtype=torch.int32, device="cuda")
     fva.fva_repair(mask, topk, g, kfloor, counts, idx, hw, wl)
+    # the fused entry point on the same inputs, with and without the route outputs
+    fused = dict(counts=torch.empty_like(counts), idx=torch.full_like(idx, -1), head_work=torch.empty_like(hw),
+                 worklist=torch.empty_like(wl), mask=torch.empty_like(mask), topk=torch.empty_like(topk))
+    fva.fva_route_repair(qr, kr, g, p, kfloor, fused["counts"], fused["idx"], fused["head_work"],
+                         fused["worklist"], ws, topp_mask=fused["mask"], topk_idx=fused["topk"])
+    bare = dict(counts=torch.empty_like(counts), idx=torch.full_like(idx, -1), head_work=torch.empty_like(hw),
+                worklist=torch.empty_like(wl))
+    fva.fva_route_repair(qr, kr, g, p, kfloor, bare["counts"], bare["idx"], bare["head_work"], bare["worklist"],
+                         ws)
     fva.fva_block_sparse_attn(qr, kr, vr, counts, idx, wl if use_lpt else None, g, 0.0, outr)
     fva.fva_inverse_reorder(outr, out, g)
     torch.cuda.synchronize()
     assert fva.fva_get_device_error() == 0
     dev.update(qr=qr, kr=kr, vr=vr, mask=mask, topk=topk, logits=logits, counts=counts, idx=idx, head_work=hw,
-               worklist=wl, outr=outr, out=out)
+               worklist=wl, outr=outr, out=out, fused=fused, bare=bare)
     return dev
+
+
+def check_fused(dev: dict):
+    """fva_route_repair gives exactly what fva_route followed by fva_repair gives."""
+    for res in (dev["fused"], dev["bare"]):
+        for key in ("counts", "head_work", "worklist"):
+            assert torch.equal(res[key], dev[key]), key
+        Nb = dev["idx"].shape[-1]
+        valid = torch.arange(Nb, device=dev["idx"].device)[None, None, None, :] < dev["counts"][..., None]
+        assert torch.equal(torch.where(valid, res["idx"], -1), torch.where(valid, dev["idx"], -1))
+    assert torch.equal(dev["fused"]["mask"], dev["mask"])
+    assert torch.equal(dev["fused"]["topk"], dev["topk"])
 
 
 def check_route(rr: O.RouteResult, mask_dev: np.ndarray, topk_dev: np.ndarray, max_tie_frac=0.02):

@@ -23,7 +23,8 @@ def _declared():
 
 def test_every_declared_symbol_is_exported():
     names = _declared()
-    assert {"fva_reorder", "fva_inverse_reorder", "fva_route", "fva_repair", "fva_block_sparse_attn"} <= names
+    assert {"fva_reorder", "fva_inverse_reorder", "fva_route", "fva_repair", "fva_route_repair",
+            "fva_block_sparse_attn"} <= names
     raw = ctypes.CDLL(fva.LIB_PATH)
     for n in sorted(names):
         assert hasattr(raw, n), n
@@ -42,12 +43,12 @@ def _g(**kw):
 
 def test_workspace_size_queries():
     g = _g()
-    # pooled Q and K (float64) plus the float64 logits, each 256-byte aligned
+    # pooled Q and K (float64), each 256-byte aligned
     nb = g.Nb
     rows = g.B * g.H * nb
     def al(x):
         return (x + 255) // 256 * 256
-    assert fva.fva_route_workspace_size(g) == 2 * al(rows * g.d * 8) + al(rows * nb * 8)
+    assert fva.fva_route_workspace_size(g) == 2 * al(rows * g.d * 8)
     assert fva.fva_repair_workspace_size(g) == 0
     assert fva.fva_route_workspace_size(_g(X=9)) == 0          # invalid geometry
 
@@ -78,6 +79,15 @@ def test_invalid_arguments_rejected_on_host():
     assert L.fva_route(*args(0.9, 1, 4096, need - 1)) == fva.FVA_ERR_INVALID_ARG
     assert b"workspace too small" in L.fva_last_error()
     assert L.fva_route(*args(0.9, 1, 4100, need)) == fva.FVA_ERR_INVALID_ARG  # not 256-aligned
+    # fused route + repair: same argument rules
+    fargs = lambda p, k, ws, wsb: (256, 512, g, p, k, None, None, 16, 32, 64, 128, ws, wsb, None)
+    assert L.fva_route_repair(*fargs(0.0, 1, 4096, need)) == fva.FVA_ERR_INVALID_ARG
+    assert L.fva_route_repair(*fargs(0.9, 0, 4096, need)) == fva.FVA_ERR_INVALID_ARG
+    assert L.fva_route_repair(*fargs(0.9, 1, 4096, need - 1)) == fva.FVA_ERR_INVALID_ARG
+    assert b"workspace too small" in L.fva_last_error()
+    assert L.fva_route_repair(256, 512, g, 0.9, 1, None, None, None, 32, 64, 128, 4096, need, None) == \
+        fva.FVA_ERR_INVALID_ARG
+    assert b"null" in L.fva_last_error()
     # repair / attention: null pointers, k, unsupported tile for attention
     assert L.fva_repair(None, 16, g, 1, 16, 16, 16, 16, None, 0, None) == fva.FVA_ERR_INVALID_ARG
     assert L.fva_repair(16, 16, g, 0, 16, 16, 16, 16, None, 0, None) == fva.FVA_ERR_INVALID_ARG

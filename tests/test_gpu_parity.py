@@ -13,7 +13,8 @@ pytestmark = pytest.mark.gpu
 
 import oracle as O
 import synth
-from gpu_util import (bf16_dev_to_f64, check_repair, check_route, compare_attention, run_path, to_bits, to_dev)
+from gpu_util import (bf16_dev_to_f64, check_fused, check_repair, check_route, compare_attention, run_path, to_bits,
+                      to_dev)
 
 
 @pytest.fixture(scope="module")
@@ -70,9 +71,10 @@ def test_path_matches_oracle(fva, name):
     if cfg.p >= 1.0:
         assert (mask_dev == 1).all()
 
-    # a5: repair, exact given the device's own route outputs
+    # a5: repair, exact given the device's own route outputs; the fused entry agrees exactly
     rp = check_repair(dev, mask_dev, topk_dev)
     assert (rp.counts >= min(cfg.k, og.Nb)).all()
+    check_fused(dev)
 
     # a6: attention with the device index lists, all items
     want = O.attention(qr, kr, vr, rp.counts, rp.idx, og.S)
@@ -81,6 +83,47 @@ def test_path_matches_oracle(fva, name):
 
     # a7: inverse reorder, bit-exact against the oracle's inverse of the device output
     assert np.array_equal(to_bits(dev["out"]), O.inverse_reorder(to_bits(dev["outr"]), og))
+
+
+# Rows wider than 256 blocks select through the wider per-lane layouts (20, 40 and 64
+# blocks per lane); routing and repair are checked in full, attention is not run.
+WIDE = {
+    "nb300_d128": _cfg("nb300_d128", H=2, T=3, Y=80, X=80, tt=1, ty=8, tx=8, seed=21),
+    "nb700_d64": _cfg("nb700_d64", H=2, d=64, T=7, Y=80, X=80, tt=1, ty=8, tx=8, seed=22),
+    "nb1500_d128": _cfg("nb1500_d128", H=1, T=15, Y=80, X=80, tt=1, ty=8, tx=8, p=0.95, k=20, seed=23),
+}
+
+
+@pytest.mark.parametrize("name", list(WIDE))
+def test_route_wide_rows(fva, name):
+    cfg = WIDE[name]
+    g = fva.Geom.of(cfg)
+    og = O.Geometry.of(cfg)
+    q, k, _ = synth.make_qkv(cfg)
+    qr, kr = O.reorder(q, og), O.reorder(k, og)
+    shp = (g.B, g.H, g.N, g.d)
+    qd, kd = to_dev(qr), to_dev(kr)
+    kk = min(cfg.k, g.Nb)
+    mask = torch.empty((g.B, g.H, g.Nb, g.Nb), dtype=torch.uint8, device="cuda")
+    topk = torch.empty((g.B, g.H, g.Nb, kk), dtype=torch.int32, device="cuda")
+    logits = torch.empty((g.B, g.H, g.Nb, g.Nb), dtype=torch.float64, device="cuda")
+    ws = torch.empty((fva.fva_route_workspace_size(g),), dtype=torch.uint8, device="cuda")
+    fva.fva_route(qd, kd, g, cfg.p, cfg.k, mask, topk, ws, logits_out=logits)
+    counts = torch.empty((g.B, g.H, g.Nb), dtype=torch.int32, device="cuda")
+    idx = torch.full((g.B, g.H, g.Nb, g.Nb), -1, dtype=torch.int32, device="cuda")
+    hw = torch.empty((g.B, g.H), dtype=torch.int64, device="cuda")
+    wl = torch.empty((g.B * g.H * g.Nb,), dtype=torch.int32, device="cuda")
+    fva.fva_route_repair(qd, kd, g, cfg.p, cfg.k, counts, idx, hw, wl, ws)
+    torch.cuda.synchronize()
+    assert fva.fva_get_device_error() == 0
+    assert shp == tuple(qd.shape)
+    rr = O.route(qr, kr, og, cfg.p, cfg.k)
+    assert np.allclose(logits.cpu().numpy(), rr.L, rtol=1e-12, atol=1e-12)
+    mask_dev, topk_dev = mask.cpu().numpy(), topk.cpu().numpy()
+    # a diffuse row of Nb blocks climbs to p in steps of about 1/Nb of the mass, so the
+    # 1e-5 band around p flags about 2e-5 * Nb of such rows (2.4 % at Nb = 700)
+    check_route(rr, mask_dev, topk_dev, max_tie_frac=0.05)
+    check_repair(dict(counts=counts, idx=idx, head_work=hw, worklist=wl), mask_dev, topk_dev)
 
 
 def test_lpt_and_static_order_identical(fva):

@@ -16,7 +16,7 @@ def _geom(fva, cfg):
 
 def test_oversized_geometry_is_rejected_without_gpu_work():
     import block_sparse_attention_44_b200 as fva
-    g = _geom(fva, synth.CONFIGS["wan720p"])           # needs ~164 MB of routing scratch
+    g = _geom(fva, synth.CONFIGS["wan720p"].with_(tt=1))   # 64-token tiles: ~94 MiB of routing scratch
     assert fva.fva_route_workspace_size(g) > fva.ROUTE_STATIC_SCRATCH_BYTES
     rc = fva.lib.fva_route_static(256, 512, g.c(), 0.9, 4, 768, 1024, None, None)
     assert rc == fva.FVA_ERR_UNSUPPORTED
