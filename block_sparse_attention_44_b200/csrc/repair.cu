@@ -9,7 +9,8 @@
 //                    diagonal, written as an ascending id list with ballot/popc.
 //   lpt_kernel     — one CTA: per-head sums, then a stable counting sort of all
 //                    items by count (descending) with per-warp histograms so it
-//                    stays deterministic.
+//                    stays deterministic; the counts are staged in shared memory
+//                    when they fit.
 #include "fva_common.cuh"
 #include "fva_internal.h"
 
@@ -55,48 +56,66 @@ __global__ void __launch_bounds__(kCompactWarps * 32) compact_kernel(const uint8
   if (lane == 0) counts[row] = pos;
 }
 
-constexpr int kLptWarps = 16;
 constexpr int kLptBatch = 8;   // counts loaded per lane before they are used
 
-// One CTA.  Items are split into kLptWarps contiguous chunks; warp w histograms its
-// chunk, so a stable scatter only needs, per count value, the number of items in
-// earlier chunks and the running position inside the warp's own chunk.
-__global__ void __launch_bounds__(kLptWarps * 32) lpt_kernel(const int32_t* __restrict__ counts, long long BH, int Nb,
-                                                             int64_t* __restrict__ head_work,
-                                                             int32_t* __restrict__ worklist) {
+// One CTA of NW warps.  Items are split into NW contiguous chunks; warp w histograms
+// its chunk, so a stable scatter only needs, per count value, the number of items in
+// earlier chunks and the running position inside the warp's own chunk.  With `staged`
+// the counts are first copied to shared memory (one pass over global memory).
+template <int NW>
+__global__ void __launch_bounds__(NW * 32) lpt_kernel(const int32_t* __restrict__ counts, long long BH, int Nb,
+                                                      int staged, int64_t* __restrict__ head_work,
+                                                      int32_t* __restrict__ worklist) {
   extern __shared__ unsigned lpt_smem[];
   const int nb1 = Nb + 1;                       // counts are in [0, Nb]
-  unsigned* hist = lpt_smem;                    // [kLptWarps][nb1], later the per-warp cursors
-  unsigned* start = lpt_smem + kLptWarps * nb1; // [nb1]: items with a larger count (descending order)
+  unsigned* hist = lpt_smem;                    // [NW][nb1], later the per-warp cursors
+  unsigned* start = lpt_smem + NW * nb1;        // [nb1]: items with a larger count (descending order)
+  int32_t* sc = reinterpret_cast<int32_t*>(start + nb1);   // [n] when staged
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x & 31;
   const long long n = BH * Nb;
-  const long long chunk = (n + kLptWarps - 1) / kLptWarps;
+  const long long chunk = (n + NW - 1) / NW;
   const long long lo = warp * chunk;
   const long long hi = min(n, lo + chunk);
 
-  for (int e = threadIdx.x; e < kLptWarps * nb1; e += blockDim.x) hist[e] = 0;
+  for (int e = threadIdx.x; e < NW * nb1; e += blockDim.x) hist[e] = 0;
+  if (staged) {
+    for (long long base = 0; base < n; base += static_cast<long long>(blockDim.x) * kLptBatch) {
+      int c[kLptBatch];
+#pragma unroll
+      for (int t = 0; t < kLptBatch; ++t) {
+        const long long u = base + threadIdx.x + static_cast<long long>(blockDim.x) * t;
+        c[t] = u < n ? __ldg(counts + u) : 0;
+      }
+#pragma unroll
+      for (int t = 0; t < kLptBatch; ++t) {
+        const long long u = base + threadIdx.x + static_cast<long long>(blockDim.x) * t;
+        if (u < n) sc[u] = c[t];
+      }
+    }
+  }
   __syncthreads();
+  const int32_t* cs = staged ? sc : counts;
   for (long long base = lo; base < hi; base += 32 * kLptBatch) {
     int c[kLptBatch];
 #pragma unroll
     for (int t = 0; t < kLptBatch; ++t) {
       const long long u = base + lane + 32 * t;
-      c[t] = u < hi ? __ldg(counts + u) : -1;
+      c[t] = u < hi ? cs[u] : -1;
     }
 #pragma unroll
     for (int t = 0; t < kLptBatch; ++t)
       if (c[t] >= 0) atomicAdd(&hist[warp * nb1 + c[t]], 1u);
   }
   // realised per-head workload
-  for (long long bh = warp; bh < BH; bh += kLptWarps) {
+  for (long long bh = warp; bh < BH; bh += NW) {
     long long s = 0;
     for (int i0 = 0; i0 < Nb; i0 += 32 * kLptBatch) {
       int c[kLptBatch];
 #pragma unroll
       for (int t = 0; t < kLptBatch; ++t) {
         const int i = i0 + lane + 32 * t;
-        c[t] = i < Nb ? __ldg(counts + bh * Nb + i) : 0;
+        c[t] = i < Nb ? cs[bh * Nb + i] : 0;
       }
 #pragma unroll
       for (int t = 0; t < kLptBatch; ++t) s += c[t];
@@ -110,7 +129,7 @@ __global__ void __launch_bounds__(kLptWarps * 32) lpt_kernel(const int32_t* __re
   for (int v = threadIdx.x; v < nb1; v += blockDim.x) {
     unsigned t = 0;
 #pragma unroll
-    for (int w = 0; w < kLptWarps; ++w) t += hist[w * nb1 + v];
+    for (int w = 0; w < NW; ++w) t += hist[w * nb1 + v];
     start[v] = t;
   }
   __syncthreads();
@@ -143,7 +162,7 @@ __global__ void __launch_bounds__(kLptWarps * 32) lpt_kernel(const int32_t* __re
   for (int v = threadIdx.x; v < nb1; v += blockDim.x) {
     unsigned run = start[v];
 #pragma unroll
-    for (int w = 0; w < kLptWarps; ++w) {
+    for (int w = 0; w < NW; ++w) {
       const unsigned t = hist[w * nb1 + v];
       hist[w * nb1 + v] = run;
       run += t;
@@ -156,7 +175,7 @@ __global__ void __launch_bounds__(kLptWarps * 32) lpt_kernel(const int32_t* __re
 #pragma unroll
     for (int t = 0; t < kLptBatch; ++t) {
       const long long u = base + lane + 32 * t;
-      c[t] = u < hi ? __ldg(counts + u) : -1;
+      c[t] = u < hi ? cs[u] : -1;
     }
 #pragma unroll
     for (int t = 0; t < kLptBatch; ++t) {
@@ -178,10 +197,23 @@ __global__ void __launch_bounds__(kLptWarps * 32) lpt_kernel(const int32_t* __re
 
 cudaError_t launch_lpt(const int32_t* counts, const Dims& D, int64_t* head_work, int32_t* worklist, cudaStream_t s,
                        int* launches) {
-  const size_t lsmem = (static_cast<size_t>(kLptWarps) + 1) * (D.Nb + 1) * sizeof(unsigned);
-  cudaError_t e = cudaFuncSetAttribute(lpt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(lsmem));
-  if (e != cudaSuccess) return e;
-  lpt_kernel<<<1, kLptWarps * 32, lsmem, s>>>(counts, D.BH(), D.Nb, head_work, worklist);
+  // 32 warps with the counts staged in shared memory when everything fits, else 16
+  // warps reading the counts from global memory
+  constexpr size_t kMaxSmem = 227 * 1024;
+  const size_t nb1 = static_cast<size_t>(D.Nb) + 1;
+  const size_t n = static_cast<size_t>(D.rows());
+  const size_t big = (32 + 1) * nb1 * sizeof(unsigned) + n * sizeof(int32_t);
+  cudaError_t e;
+  if (big <= kMaxSmem) {
+    e = cudaFuncSetAttribute(lpt_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(big));
+    if (e != cudaSuccess) return e;
+    lpt_kernel<32><<<1, 32 * 32, big, s>>>(counts, D.BH(), D.Nb, 1, head_work, worklist);
+  } else {
+    const size_t small = (16 + 1) * nb1 * sizeof(unsigned);
+    e = cudaFuncSetAttribute(lpt_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(small));
+    if (e != cudaSuccess) return e;
+    lpt_kernel<16><<<1, 16 * 32, small, s>>>(counts, D.BH(), D.Nb, 0, head_work, worklist);
+  }
   ++*launches;
   return cudaGetLastError();
 }

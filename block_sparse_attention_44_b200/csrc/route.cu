@@ -12,23 +12,29 @@
 //                   the FP64 tensor path (mma.sync m8n8k4), then one warp per row:
 //                   softmax, Top-p boundary, Top-k floor, outputs (mask, floor ids,
 //                   logits, compacted kept list).
-// The heads are split into chunks: chunk c is pooled on the caller's stream while a
-// second stream scores and selects chunk c - 1, so selection runs under the memory
-// stream instead of after it.  The two streams meet through events only.
+// Both run on the caller's stream, one after the other.  (Splitting the heads into
+// chunks and selecting chunk c on a second stream while chunk c + 1 is pooled was
+// measured slower: the two kernels compete for the same SM registers and issue slots,
+// and the per-chunk grids lose their wave tails.)
 //
 // Selection arithmetic (deterministic, exact integer sums):
-//   - softmax weights e_j = exp(L_ij - max_j L_ij) in float64, then the mass
-//     m_j = floor(e_j / z * 2^31) (z = sum_j e_j) as an unsigned integer;
+//   - softmax weights e_j = 2^((L_ij - max_j L_ij) log2 e) in float32 (the float64
+//     difference rounded once, then the hardware base-2 exponential), z = sum_j e_j
+//     pairwise in float32, and the mass m_j = floor(e_j * (2^31 / z)) as an integer;
 //   - the Top-p boundary is the first position, in the ranking (logit descending,
 //     block id ascending), where the running sum of m reaches ceil(p * 2^31): found
 //     by a 14-step bisection over the bucket index q_j = floor((max L - L_ij) * 256)
 //     (buckets 1/256 logit wide rank like the logits; warp sums by redux.sync), then
 //     inside the boundary bucket by the exact float64 logits;
-//   - the Top-k floor by repeated warp argmax over (logit, -block id).
-// Every mass carries a relative error below 2e-7 and is truncated by less than 2^-31,
-// so the running sum at any cut is within 1.2e-6 of the exact cumulative softmax
-// mass: a kept set can differ from the exact one only where the cumulative mass at
-// the cut lies within that distance of p.
+//   - the Top-k floor by repeated warp argmax over (logit, -block id); argmaxes are
+//     three integer warp reductions over an order-preserving key of the float64 logit,
+//     so every ranking decision is exact.
+// Error of the running mass at any cut against the exact cumulative softmax mass:
+// rounding of the exponent argument (|x| <= 65, 2^-24 relative) weighted by the masses
+// <= 5e-7, the exponential (2^-22 relative) 2.4e-7, z (pairwise, 8 levels) 4.8e-7, the
+// scaling 1.2e-7, truncation Nb * 2^-31 <= 1e-6: in all below 2.5e-6.  A kept set can
+// differ from the exact one only where the cumulative mass at the cut lies that close
+// to p (rows the parity rule flags as ties, whose band is 1e-5).
 #include <limits.h>
 #include <math.h>
 
@@ -41,7 +47,6 @@ namespace {
 constexpr int kRouteThreads = 256;
 constexpr int kRouteWarps = kRouteThreads / 32;
 constexpr int kPoolThreads = 256;
-constexpr int kMaxChunks = 4;           // head chunks overlapped across the two streams
 constexpr unsigned kQCap = 45u * 256u;  // bucket of blocks whose weight e^(L - max) < e^-45 (mass 0)
 constexpr unsigned kQPad = 0xFFFFu;     // bucket of the padding columns past Nb
 constexpr unsigned kFull = 0xffffffffu;
@@ -70,35 +75,34 @@ __device__ __forceinline__ void bf16x8_to_f64_add(const uint4& v, double (&acc)[
   }
 }
 
-__device__ __forceinline__ double warp_max_f64(double v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmax(v, __shfl_xor_sync(kFull, v, o));
-  return v;
+typedef unsigned long long u64;
+
+// Order-preserving map of a float64 logit to an unsigned key (larger logit -> larger
+// key, -0 and +0 equal); key 0 lies below every finite logit and is used for "none".
+__device__ __forceinline__ u64 order_key(double L) {
+  if (L == 0.0) L = 0.0;
+  const u64 u = static_cast<u64>(__double_as_longlong(L));
+  return (u & 0x8000000000000000ull) ? ~u : (u | 0x8000000000000000ull);
 }
-__device__ __forceinline__ double warp_sum_f64(double v) {
+__device__ __forceinline__ double key_value(u64 k) {
+  const u64 u = (k & 0x8000000000000000ull) ? (k & 0x7FFFFFFFFFFFFFFFull) : ~k;
+  return __longlong_as_double(static_cast<long long>(u));
+}
+
+// Warp-wide best (key descending, t ascending) with three integer warp reductions;
+// every lane returns the winning key and t (key 0 if no lane had a candidate).
+__device__ __forceinline__ void warp_best(u64 key, unsigned t, u64& bkey, unsigned& bt) {
+  const unsigned khi = static_cast<unsigned>(key >> 32), klo = static_cast<unsigned>(key);
+  const unsigned hi = __reduce_max_sync(kFull, khi);
+  const unsigned lo = __reduce_max_sync(kFull, khi == hi ? klo : 0u);
+  bt = __reduce_min_sync(kFull, (khi == hi && klo == lo) ? t : 0xFFFFFFFFu);
+  bkey = (static_cast<u64>(hi) << 32) | lo;
+}
+
+__device__ __forceinline__ float warp_sum_f32(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
   return v;
-}
-
-// (L, t) ranks before (L2, t2): logit descending, block id ascending.
-__device__ __forceinline__ bool ranks_before(double L, int t, double L2, int t2) {
-  return L > L2 || (L == L2 && t < t2);
-}
-
-// Warp argmax of (L, t) in ranking order, carrying a payload word.
-__device__ __forceinline__ void warp_argmax(double& L, int& t, unsigned& w) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const double oL = __shfl_xor_sync(kFull, L, o);
-    const int ot = __shfl_xor_sync(kFull, t, o);
-    const unsigned ow = __shfl_xor_sync(kFull, w, o);
-    if (ranks_before(oL, ot, L, t)) {
-      L = oL;
-      t = ot;
-      w = ow;
-    }
-  }
 }
 
 // ------------------------------------------------------------------ pooling -------
@@ -155,70 +159,88 @@ __device__ __forceinline__ unsigned bisect(const unsigned (&q)[PL], const unsign
 }
 
 // Walks bucket qs in ranking order from weight `acc` (the weight of every better
-// bucket) until the running weight reaches T; returns that block's (logit, id).
+// bucket) until the running weight reaches T; returns that block's (key, id).
+// Kr = the row's order keys in shared memory.
 template <int PL, bool BY_MASS>
-__device__ __forceinline__ void walk_bucket(const double* Lr, const unsigned (&q)[PL], const unsigned (&m)[PL], unsigned qs,
-                            unsigned acc, unsigned T, double& Lb, int& jb) {
+__device__ __forceinline__ void walk_bucket(const u64* Kr, const unsigned (&q)[PL], const unsigned (&m)[PL],
+                                            unsigned qs, unsigned acc, unsigned T, u64& kb, int& jb) {
   const int lane = threadIdx.x & 31;
-  double Lp = INFINITY;
-  int jp = -1;
+  u64 pkey = ~0ull;          // the last block taken, as (key, id); none yet
+  unsigned pt = 0;
   for (int guard = 0; guard < 32 * PL; ++guard) {
-    double bL = -INFINITY;
-    int bt = INT_MAX;
-    unsigned bw = 0;
+    u64 bk = 0;
+    unsigned bt = 0xFFFFFFFFu, bw = 0;
 #pragma unroll
     for (int s = 0; s < PL; ++s) {
       if (q[s] != qs) continue;
-      const int t = lane + 32 * s;
-      const double L = Lr[t];
-      if (ranks_before(Lp, jp, L, t) && ranks_before(L, t, bL, bt)) {
-        bL = L;
+      const unsigned t = lane + 32 * s;
+      const u64 k = Kr[t];
+      const bool after = k < pkey || (k == pkey && t > pt);
+      if (after && k > bk) {   // t ascends with s: the first of equal keys is kept
+        bk = k;
         bt = t;
         bw = BY_MASS ? m[s] : 1u;
       }
     }
-    warp_argmax(bL, bt, bw);
-    if (bt == INT_MAX) break;   // bucket exhausted: cannot happen when the bucket reaches T
-    acc += bw;
+    u64 wk;
+    unsigned wt;
+    warp_best(bk, bt, wk, wt);
+    if (wk == 0) break;        // bucket exhausted: cannot happen when the bucket reaches T
+    acc += __shfl_sync(kFull, bw, wt & 31);
     if (acc >= T) {
-      Lb = bL;
-      jb = bt;
+      kb = wk;
+      jb = static_cast<int>(wt);
       return;
     }
-    Lp = bL;
-    jp = bt;
+    pkey = wk;
+    pt = wt;
   }
-  Lb = -INFINITY;   // keep everything
+  kb = 0;   // keep everything
   jb = INT_MAX;
 }
 
-// Row i of (b, h) = bh; Lr = its logits in shared memory (32*PL entries, -inf past Nb).
+// Block (key k, id t) ranks at or before the boundary (kb, jb).
+__device__ __forceinline__ bool at_or_before(u64 k, int t, u64 kb, int jb) {
+  return k > kb || (k == kb && t <= jb);
+}
+
+// Row i of (b, h) = bh; Lr = its logits in shared memory (32*PL entries, -inf past Nb),
+// replaced in place by their order keys once the weights are taken.
 template <int PL>
-__device__ __forceinline__ void select_row(const RouteArgs& a, long long bh, int i, const double* Lr) {
+__device__ __forceinline__ void select_row(const RouteArgs& a, long long bh, int i, double* Lr) {
   const int lane = threadIdx.x & 31;
   const int Nb = a.Nb;
   const long long row = bh * Nb + i;
 
-  double mx = -INFINITY;
+  double lmax = -INFINITY;
 #pragma unroll
-  for (int s = 0; s < PL; ++s) mx = fmax(mx, Lr[lane + 32 * s]);
-  mx = warp_max_f64(mx);
+  for (int s = 0; s < PL; ++s) lmax = fmax(lmax, Lr[lane + 32 * s]);
+  u64 mk;
+  unsigned mt;
+  warp_best(order_key(lmax), 0u, mk, mt);
+  const double mx = key_value(mk);
 
-  // weights, bucket indices; e^-45 < 2^-64: those blocks carry mass 0 and go to kQCap
+  // weights 2^((L - max) log2 e) on the MUFU unit, summed pairwise in float32; blocks
+  // more than 45 below the max (weight < e^-45, mass 0) go to bucket kQCap
   unsigned q[PL], m[PL];
-  double z = 0.0;
+  float zl = 0.0f;
+  unsigned qlive = 0;
+  u64* Kr = reinterpret_cast<u64*>(Lr);
 #pragma unroll
   for (int s = 0; s < PL; ++s) {
     const int t = lane + 32 * s;
-    const double d = Lr[t] - mx;
+    const double L = Lr[t];
+    const double d = L - mx;
     const bool live = d > -45.0;
-    const double e = live ? exp(d) : 0.0;
-    z += e;
-    m[s] = __float_as_uint(__double2float_rn(e));
+    const float e = live ? ex2_approx(__double2float_rn(d * 1.4426950408889634)) : 0.0f;
+    zl += e;
+    m[s] = __float_as_uint(e);
     q[s] = live ? static_cast<unsigned>(-d * 256.0) : (t < Nb ? kQCap : kQPad);
+    if (live) qlive = max(qlive, q[s]);
+    Kr[t] = order_key(L);    // this lane's own slot: no other lane reads it before the swap
   }
-  z = warp_sum_f64(z);
-  const float scale = __double2float_rn(0x1p31 / z);
+  const float z = warp_sum_f32(zl);
+  const float scale = __fdiv_rn(0x1p31f, z);
   unsigned part = 0;
 #pragma unroll
   for (int s = 0; s < PL; ++s) {
@@ -226,54 +248,84 @@ __device__ __forceinline__ void select_row(const RouteArgs& a, long long bh, int
     part += m[s];
   }
   const unsigned tot = __reduce_add_sync(kFull, part);
+  qlive = __reduce_max_sync(kFull, qlive);
 
-  // Top-p boundary (Lp_b, jp_b): the kept set is every block ranking at or before it
+  // Top-p boundary (kpb, jpb): the kept set is every block ranking at or before it
   const bool all_p = a.keep_all_p || tot < a.target;
   unsigned qp = 0;
-  double Lpb = -INFINITY;
+  u64 kpb = 0;
   int jpb = INT_MAX;
   if (!all_p) {
-    qp = bisect<PL, true>(q, m, 0u, kQCap - 1u, a.target);
+    qp = bisect<PL, true>(q, m, 0u, qlive, a.target);
     unsigned above = 0;
 #pragma unroll
     for (int s = 0; s < PL; ++s)
       if (q[s] < qp) above += m[s];
     above = __reduce_add_sync(kFull, above);
-    walk_bucket<PL, true>(Lr, q, m, qp, above, a.target, Lpb, jpb);
+    walk_bucket<PL, true>(Kr, q, m, qp, above, a.target, kpb, jpb);
   }
 
-  // Top-k floor
+  // Top-k floor: bit s of `taken` marks block lane + 32 s (kk <= kTopkArgmaxMax)
   const int kk = a.kk;
-  unsigned long long taken = 0;   // bit s: block lane + 32 s is in the floor (kk <= kTopkArgmaxMax)
+  unsigned long long taken = 0;
   unsigned qk = 0;
-  double Lkb = -INFINITY;
+  u64 kkb = 0;
   int jkb = INT_MAX;
   int32_t* krow = a.topk_idx ? a.topk_idx + row * kk : nullptr;
-  if (kk <= kTopkArgmaxMax) {
-    int mine = INT_MAX;   // lane c holds the c-th chosen id
+  unsigned mine = 0xFFFFFFFFu;   // lane c holds the c-th chosen id
+  if (kk <= 4) {
+    // each lane's four best (key descending, id ascending) in one pass, then four
+    // warp-wide picks among the lane heads
+    u64 k4[4] = {0, 0, 0, 0};
+    unsigned s4[4] = {0, 0, 0, 0};
+#pragma unroll
+    for (int s = 0; s < PL; ++s) {
+      const u64 k = lane + 32 * s < Nb ? Kr[lane + 32 * s] : 0ull;
+      const bool c0 = k > k4[0], c1 = k > k4[1], c2 = k > k4[2], c3 = k > k4[3];
+      k4[3] = c2 ? k4[2] : (c3 ? k : k4[3]);
+      s4[3] = c2 ? s4[2] : (c3 ? s : s4[3]);
+      k4[2] = c1 ? k4[1] : (c2 ? k : k4[2]);
+      s4[2] = c1 ? s4[1] : (c2 ? s : s4[2]);
+      k4[1] = c0 ? k4[0] : (c1 ? k : k4[1]);
+      s4[1] = c0 ? s4[0] : (c1 ? s : s4[1]);
+      k4[0] = c0 ? k : k4[0];
+      s4[0] = c0 ? s : s4[0];
+    }
     for (int c = 0; c < kk; ++c) {
-      double bL = -INFINITY;
-      int bt = INT_MAX;
-      unsigned bs = 0;
+      u64 wk;
+      unsigned wt;
+      warp_best(k4[0], static_cast<unsigned>(lane) + 32u * s4[0], wk, wt);
+      if ((wt & 31u) == static_cast<unsigned>(lane)) {   // the winner lane pops its head
+        taken |= 1ull << s4[0];
+        k4[0] = k4[1];
+        s4[0] = s4[1];
+        k4[1] = k4[2];
+        s4[1] = s4[2];
+        k4[2] = k4[3];
+        s4[2] = s4[3];
+        k4[3] = 0;
+      }
+      if (lane == c) mine = wt;
+    }
+  } else if (kk <= kTopkArgmaxMax) {
+    for (int c = 0; c < kk; ++c) {
+      u64 bk = 0;
+      unsigned bt = 0xFFFFFFFFu;
 #pragma unroll
       for (int s = 0; s < PL; ++s) {
         const int t = lane + 32 * s;
         if (((taken >> s) & 1ull) || t >= Nb) continue;
-        const double L = Lr[t];
-        if (ranks_before(L, t, bL, bt)) {
-          bL = L;
+        const u64 k = Kr[t];
+        if (k > bk) {
+          bk = k;
           bt = t;
-          bs = static_cast<unsigned>(s);
         }
       }
-      warp_argmax(bL, bt, bs);
-      if ((bt & 31) == lane) taken |= 1ull << bs;
-      if (lane == c) mine = bt;
-    }
-    if (krow) {   // ascending block id: lane c writes its id at its rank
-      int rank = 0;
-      for (int c = 0; c < kk; ++c) rank += __shfl_sync(kFull, mine, c) < mine ? 1 : 0;
-      if (lane < kk) krow[rank] = mine;
+      u64 wk;
+      unsigned wt;
+      warp_best(bk, bt, wk, wt);
+      if ((wt & 31u) == static_cast<unsigned>(lane)) taken |= 1ull << (wt >> 5);
+      if (lane == c) mine = wt;
     }
   } else {
     qk = bisect<PL, false>(q, m, 0u, kQCap, static_cast<unsigned>(kk));
@@ -282,37 +334,65 @@ __device__ __forceinline__ void select_row(const RouteArgs& a, long long bh, int
     for (int s = 0; s < PL; ++s)
       if (q[s] < qk) ++above;
     above = __reduce_add_sync(kFull, above);
-    walk_bucket<PL, false>(Lr, q, m, qk, above, static_cast<unsigned>(kk), Lkb, jkb);
+    walk_bucket<PL, false>(Kr, q, m, qk, above, static_cast<unsigned>(kk), kkb, jkb);
+  }
+  const bool big_k = kk > kTopkArgmaxMax;
+  if (krow && !big_k) {   // ascending block id: lane c writes its id at its rank
+    int rank = 0;
+    for (int c = 0; c < kk; ++c) rank += __shfl_sync(kFull, mine, c) < mine ? 1 : 0;
+    if (lane < kk) krow[rank] = static_cast<int32_t>(mine);
   }
 
-  // outputs: Top-p mask, floor ids (large floors), logits, compacted kept list
-  uint8_t* mrow = a.topp_mask ? a.topp_mask + row * Nb : nullptr;
-  double* lrow = a.logits_out ? a.logits_out + row * Nb : nullptr;
-  int32_t* irow = a.counts ? a.idx + row * Nb : nullptr;
-  const bool big_k = kk > kTopkArgmaxMax;
-  int kpos = 0, pos = 0;
+  // membership bits of this lane's blocks: Top-p set, floor
+  unsigned long long inp = 0, ink = taken;
 #pragma unroll
   for (int s = 0; s < PL; ++s) {
-    if (32 * s >= Nb) break;
     const int t = lane + 32 * s;
-    const bool valid = t < Nb;
-    const double L = Lr[t];
-    const bool in_p = valid && (all_p || q[s] < qp || (q[s] == qp && !ranks_before(Lpb, jpb, L, t)));
-    const bool in_k = big_k ? valid && (q[s] < qk || (q[s] == qk && !ranks_before(Lkb, jkb, L, t)))
-                            : ((taken >> s) & 1ull) != 0;
-    if (valid && mrow) mrow[t] = in_p ? 1 : 0;
-    if (valid && lrow) lrow[t] = L;
-    if (big_k) {
-      const unsigned bal = __ballot_sync(kFull, in_k);
-      if (in_k && krow) krow[kpos + __popc(bal & ((1u << lane) - 1u))] = t;
-      kpos += __popc(bal);
-    }
-    if (irow) {
-      const bool keep = in_p || in_k || t == i;
-      const unsigned bal = __ballot_sync(kFull, valid && keep);
-      if (valid && keep) irow[pos + __popc(bal & ((1u << lane) - 1u))] = t;
+    bool in = all_p || q[s] < qp;
+    if (!all_p && q[s] == qp) in = at_or_before(Kr[t], t, kpb, jpb);
+    if (in && t < Nb) inp |= 1ull << s;
+    if (big_k && t < Nb && (q[s] < qk || (q[s] == qk && at_or_before(Kr[t], t, kkb, jkb)))) ink |= 1ull << s;
+  }
+
+  // outputs: compacted kept list, Top-p mask, floor ids (large floors), logits
+  const int nsl = (Nb + 31) / 32;   // slots holding blocks
+  int32_t* irow = a.counts ? a.idx + row * Nb : nullptr;
+  int pos = 0;
+  if (irow) {
+    const unsigned long long keep = inp | ink | ((i & 31) == lane ? 1ull << (i >> 5) : 0ull);
+    const unsigned lt = (1u << lane) - 1u;
+#pragma unroll
+    for (int s = 0; s < PL; ++s) {
+      if (s >= nsl) break;
+      const bool kp = (keep >> s) & 1ull;
+      const unsigned bal = __ballot_sync(kFull, kp);
+      if (kp) irow[pos + __popc(bal & lt)] = lane + 32 * s;
       pos += __popc(bal);
     }
+  }
+  if (a.topp_mask) {
+    uint8_t* mrow = a.topp_mask + row * Nb;
+#pragma unroll
+    for (int s = 0; s < PL; ++s)
+      if (lane + 32 * s < Nb) mrow[lane + 32 * s] = static_cast<uint8_t>((inp >> s) & 1ull);
+  }
+  if (big_k && krow) {
+    int kpos = 0;
+    const unsigned lt = (1u << lane) - 1u;
+#pragma unroll
+    for (int s = 0; s < PL; ++s) {
+      if (s >= nsl) break;
+      const bool kp = (ink >> s) & 1ull;
+      const unsigned bal = __ballot_sync(kFull, kp);
+      if (kp) krow[kpos + __popc(bal & lt)] = lane + 32 * s;
+      kpos += __popc(bal);
+    }
+  }
+  if (a.logits_out) {
+    double* lrow = a.logits_out + row * Nb;
+#pragma unroll
+    for (int s = 0; s < PL; ++s)
+      if (lane + 32 * s < Nb) lrow[lane + 32 * s] = key_value(Kr[lane + 32 * s]);
   }
   if (irow && lane == 0) a.counts[row] = pos;
 }
@@ -336,48 +416,65 @@ __device__ __forceinline__ void select_item(const RouteArgs& a, long long bh, in
   }
   __syncthreads();
 
-  // L = Qbar Kbar^T / sqrt(D): warp w takes column tiles w, w + 8, w + 16, ... four at
-  // a time, so each A fragment feeds four independent accumulation chains.  Fragment
-  // coordinates of m8n8k4 (row.col): A[gid][tq], B[tq][gid], C[gid][2 tq + e].
-  static_assert(R == 8, "one 8-row MMA tile per item");
+  // L = Qbar Kbar^T / sqrt(D): warp w takes column tiles w, w + 8, w + 16, ... NG at a
+  // time for all MT row tiles, so every loaded fragment feeds MT (A: NG) products and
+  // the warp runs MT * NG independent accumulation chains.  Fragment coordinates of
+  // m8n8k4 (row.col): A[gid][kq], B[kq][gid], C[gid][2 tq + e], where the four k of
+  // one product are taken as 8 c + 2 tq + h (h = 0 for the first product of a pair,
+  // 1 for the second), so each thread loads its two k of a pair as one 16-byte word.
+  // The product covers every k exactly once, in a different grouping (float64 sums).
+  // Columns past Nb read block 0 and are overwritten by -inf below.
+  constexpr int MT = R / 8;                      // 8-row tiles
+  constexpr int NG = 4 / MT;                     // column tiles per group
   constexpr int NTW = NT / kRouteWarps;          // column tiles per warp
+  static_assert(R % 8 == 0 && MT * NG == 4, "8 or 16 rows per item");
   const int gid = lane >> 2, tq = lane & 3;
   const int ntv = (Nb + 7) / 8;
-  const double rs = sqrt(static_cast<double>(D));
-  const double* qa = Qs + gid * LDQ + tq;
+  const double inv_rs = 1.0 / sqrt(static_cast<double>(D));
+  const double* qa = Qs + gid * LDQ + 2 * tq;
 #pragma unroll 1
-  for (int j0 = 0; j0 < NTW; j0 += 4) {
-    double acc[4][2];
-    const double* kp[4];
-    bool jv[4];
+  for (int j0 = 0; j0 < NTW; j0 += NG) {
+    double acc[NG][MT][2];
+    const double2* kp[NG];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < NG; ++u) {
       const int nt = warp + kRouteWarps * (j0 + u);
       const int j = nt * 8 + gid;
-      jv[u] = j0 + u < NTW && nt < ntv && j < Nb;
-      kp[u] = kb + static_cast<long long>(jv[u] ? j : 0) * D + tq;
-      acc[u][0] = acc[u][1] = 0.0;
+      const bool jv = j0 + u < NTW && nt < ntv && j < Nb;
+      kp[u] = reinterpret_cast<const double2*>(kb + static_cast<long long>(jv ? j : 0) * D + 2 * tq);
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) acc[u][mt][0] = acc[u][mt][1] = 0.0;
     }
 #pragma unroll KU
-    for (int k = 0; k < D; k += 4) {
-      const double av = qa[k];
+    for (int c = 0; c < D / 8; ++c) {
+      double2 av[MT];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const double b = jv[u] ? __ldcg(kp[u] + k) : 0.0;
-        asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
-                     : "+d"(acc[u][0]), "+d"(acc[u][1])
-                     : "d"(av), "d"(b));
+      for (int mt = 0; mt < MT; ++mt) av[mt] = *reinterpret_cast<const double2*>(qa + mt * 8 * LDQ + 8 * c);
+#pragma unroll
+      for (int u = 0; u < NG; ++u) {
+        const double2 b = __ldcg(kp[u] + 4 * c);
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+                       : "+d"(acc[u][mt][0]), "+d"(acc[u][mt][1])
+                       : "d"(av[mt].x), "d"(b.x));
+          asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+                       : "+d"(acc[u][mt][0]), "+d"(acc[u][mt][1])
+                       : "d"(av[mt].y), "d"(b.y));
+        }
       }
     }
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < NG; ++u) {
       if (j0 + u >= NTW) break;
       const int nt = warp + kRouteWarps * (j0 + u);
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int c = nt * 8 + 2 * tq + e;
-        Ls[gid * LDL + c] = c < Nb ? acc[u][e] / rs : -INFINITY;
-      }
+      for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int cc = nt * 8 + 2 * tq + e;
+          Ls[(mt * 8 + gid) * LDL + cc] = cc < Nb ? acc[u][mt][e] * inv_rs : -INFINITY;
+        }
     }
   }
   __syncthreads();
@@ -413,37 +510,6 @@ Carve carve(const Dims& D, void* ws) {
   return Carve{reinterpret_cast<double*>(w), reinterpret_cast<double*>(w + pooled)};
 }
 
-// The second stream and the fork/join events, per host thread and device (a thread
-// never shares them, so concurrent callers on other threads cannot interleave).
-struct SideStream {
-  cudaStream_t stream = nullptr;
-  cudaEvent_t ev[kMaxChunks + 2] = {};
-  bool ready = false;
-};
-
-cudaError_t side_stream(SideStream** out) {
-  thread_local SideStream ctx[64];
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  SideStream& c = ctx[dev];
-  if (!c.ready) {
-    int lo = 0, hi = 0;
-    e = cudaDeviceGetStreamPriorityRange(&lo, &hi);
-    if (e != cudaSuccess) return e;
-    e = cudaStreamCreateWithPriority(&c.stream, cudaStreamNonBlocking, hi);   // selection first when both wait
-    if (e != cudaSuccess) return e;
-    for (auto& ev : c.ev) {
-      e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming);
-      if (e != cudaSuccess) return e;
-    }
-    c.ready = true;
-  }
-  *out = &c;
-  return cudaSuccess;
-}
-
 template <int D, int PL, int R, int MINB>
 cudaError_t launch_select_variant(const RouteArgs& a, long long bh0, long long nbh, cudaStream_t s) {
   auto kern = select_kernel<D, PL, R, MINB>;
@@ -458,8 +524,8 @@ cudaError_t launch_select_variant(const RouteArgs& a, long long bh0, long long n
 template <int D>
 cudaError_t launch_select(const RouteArgs& a, long long bh0, long long nbh, cudaStream_t s) {
   if (a.Nb <= 256) return launch_select_variant<D, 8, 8, 4>(a, bh0, nbh, s);
-  if (a.Nb <= 640) return launch_select_variant<D, 20, 8, 3>(a, bh0, nbh, s);
-  if (a.Nb <= 1280) return launch_select_variant<D, 40, 8, 2>(a, bh0, nbh, s);
+  if (a.Nb <= 640) return launch_select_variant<D, 20, 16, 2>(a, bh0, nbh, s);
+  if (a.Nb <= 1280) return launch_select_variant<D, 40, 16, 1>(a, bh0, nbh, s);
   return launch_select_variant<D, 64, 8, 1>(a, bh0, nbh, s);
 }
 
@@ -488,36 +554,20 @@ cudaError_t launch_route(const void* qr, const void* kr, const Dims& D, double p
   const double tp = ceil(p * 0x1p31);
   a.target = a.keep_all_p ? 0u : static_cast<unsigned>(tp < 1.0 ? 1.0 : tp);
 
-  SideStream* side = nullptr;
-  cudaError_t e = side_stream(&side);
+  const long long rows = D.rows();
+  const dim3 pgrid(static_cast<unsigned>(2 * rows));
+  if (D.d == 128)
+    pool_kernel<128><<<pgrid, kPoolThreads, 0, s>>>(static_cast<const uint4*>(qr), static_cast<const uint4*>(kr),
+                                                    c.qbar, c.kbar, 0, rows, D.S);
+  else
+    pool_kernel<64><<<pgrid, kPoolThreads, 0, s>>>(static_cast<const uint4*>(qr), static_cast<const uint4*>(kr),
+                                                   c.qbar, c.kbar, 0, rows, D.S);
+  ++*launches;
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const long long BH = D.BH();
-  const int nchunks = static_cast<int>(BH < kMaxChunks ? BH : kMaxChunks);
-  // fork: the side stream starts after everything already queued on s
-  if ((e = cudaEventRecord(side->ev[0], s)) != cudaSuccess) return e;
-  if ((e = cudaStreamWaitEvent(side->stream, side->ev[0], 0)) != cudaSuccess) return e;
-  for (int ch = 0; ch < nchunks; ++ch) {
-    const long long bh0 = BH * ch / nchunks, bh1 = BH * (ch + 1) / nchunks;
-    const long long row0 = bh0 * D.Nb, nrows = (bh1 - bh0) * D.Nb;
-    const dim3 pgrid(static_cast<unsigned>(2 * nrows));
-    if (D.d == 128)
-      pool_kernel<128><<<pgrid, kPoolThreads, 0, s>>>(static_cast<const uint4*>(qr), static_cast<const uint4*>(kr),
-                                                      c.qbar, c.kbar, row0, nrows, D.S);
-    else
-      pool_kernel<64><<<pgrid, kPoolThreads, 0, s>>>(static_cast<const uint4*>(qr), static_cast<const uint4*>(kr),
-                                                     c.qbar, c.kbar, row0, nrows, D.S);
-    ++*launches;
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if ((e = cudaEventRecord(side->ev[ch + 1], s)) != cudaSuccess) return e;
-    if ((e = cudaStreamWaitEvent(side->stream, side->ev[ch + 1], 0)) != cudaSuccess) return e;
-    e = D.d == 128 ? launch_select<128>(a, bh0, bh1 - bh0, side->stream)
-                   : launch_select<64>(a, bh0, bh1 - bh0, side->stream);
-    ++*launches;
-    if (e != cudaSuccess) return e;
-  }
-  // join: later work on s sees every selection
-  if ((e = cudaEventRecord(side->ev[kMaxChunks + 1], side->stream)) != cudaSuccess) return e;
-  return cudaStreamWaitEvent(s, side->ev[kMaxChunks + 1], 0);
+  e = D.d == 128 ? launch_select<128>(a, 0, D.BH(), s) : launch_select<64>(a, 0, D.BH(), s);
+  ++*launches;
+  return e;
 }
 
 }  // namespace fva

@@ -87,11 +87,7 @@ size_t fva_route_workspace_size(fva_geom g);
  * sum, so the result is deterministic and the cumulative mass at any cut is within
  * 1.2e-6 of the exact one (a kept set differs from the exact rule only where the
  * cumulative mass at the cut lies that close to p).  Requires Nb <= 2048.
- * Launches: per head chunk (up to 4) a pooling kernel on `stream` and a selection
- * kernel on a second stream the library owns (one per host thread and device), so the
- * selection of a chunk runs while the next chunk is pooled; the second stream starts
- * after the work already queued on `stream` and `stream` waits for it before the call
- * returns (events), so everything stays ordered on `stream`, graph capture included.
+ * Two kernel launches on `stream`: pooling, then scoring and selection.
  */
 int fva_route(const void* qr, const void* kr, fva_geom g, double p, int32_t k,
               uint8_t* topp_mask, int32_t* topk_idx, double* logits_out,
