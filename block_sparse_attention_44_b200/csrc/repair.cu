@@ -7,10 +7,8 @@
 //
 //   compact_kernel — one warp per (b, h, i) row: kept = Top-p mask | Top-k floor |
 //                    diagonal, written as an ascending id list with ballot/popc.
-//   lpt_kernel     — one CTA: per-head sums, then a stable counting sort of all
-//                    items by count (descending) with per-warp histograms so it
-//                    stays deterministic; the counts are staged in shared memory
-//                    when they fit.
+//   lpt_kernel     — one CTA per count value (stable counting sort by count,
+//                    descending, without atomics) plus one CTA per head for W_h.
 #include "fva_common.cuh"
 #include "fva_internal.h"
 
@@ -56,164 +54,85 @@ __global__ void __launch_bounds__(kCompactWarps * 32) compact_kernel(const uint8
   if (lane == 0) counts[row] = pos;
 }
 
-constexpr int kLptBatch = 8;   // counts loaded per lane before they are used
+constexpr int kLptThreads = 256;
 
-// One CTA of NW warps.  Items are split into NW contiguous chunks; warp w histograms
-// its chunk, so a stable scatter only needs, per count value, the number of items in
-// earlier chunks and the running position inside the warp's own chunk.  With `staged`
-// the counts are first copied to shared memory (one pass over global memory).
-template <int NW>
-__global__ void __launch_bounds__(NW * 32) lpt_kernel(const int32_t* __restrict__ counts, long long BH, int Nb,
-                                                      int staged, int64_t* __restrict__ head_work,
-                                                      int32_t* __restrict__ worklist) {
-  extern __shared__ unsigned lpt_smem[];
-  const int nb1 = Nb + 1;                       // counts are in [0, Nb]
-  unsigned* hist = lpt_smem;                    // [NW][nb1], later the per-warp cursors
-  unsigned* start = lpt_smem + NW * nb1;        // [nb1]: items with a larger count (descending order)
-  int32_t* sc = reinterpret_cast<int32_t*>(start + nb1);   // [n] when staged
-  const int warp = threadIdx.x / 32;
-  const int lane = threadIdx.x & 31;
-  const long long n = BH * Nb;
-  const long long chunk = (n + NW - 1) / NW;
-  const long long lo = warp * chunk;
-  const long long hi = min(n, lo + chunk);
-
-  for (int e = threadIdx.x; e < NW * nb1; e += blockDim.x) hist[e] = 0;
-  if (staged) {
-    for (long long base = 0; base < n; base += static_cast<long long>(blockDim.x) * kLptBatch) {
-      int c[kLptBatch];
+// Block-wide exclusive prefix sum of v (every thread of a kLptThreads CTA calls it);
+// returns the exclusive prefix and the total in *total.
+__device__ __forceinline__ unsigned block_exclusive_scan(unsigned v, unsigned* total, unsigned* sh) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  unsigned incl = v;
 #pragma unroll
-      for (int t = 0; t < kLptBatch; ++t) {
-        const long long u = base + threadIdx.x + static_cast<long long>(blockDim.x) * t;
-        c[t] = u < n ? __ldg(counts + u) : 0;
-      }
-#pragma unroll
-      for (int t = 0; t < kLptBatch; ++t) {
-        const long long u = base + threadIdx.x + static_cast<long long>(blockDim.x) * t;
-        if (u < n) sc[u] = c[t];
-      }
-    }
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
   }
+  if (lane == 31) sh[warp] = incl;
   __syncthreads();
-  const int32_t* cs = staged ? sc : counts;
-  for (long long base = lo; base < hi; base += 32 * kLptBatch) {
-    int c[kLptBatch];
+  unsigned before = 0, all = 0;
 #pragma unroll
-    for (int t = 0; t < kLptBatch; ++t) {
-      const long long u = base + lane + 32 * t;
-      c[t] = u < hi ? cs[u] : -1;
-    }
-#pragma unroll
-    for (int t = 0; t < kLptBatch; ++t)
-      if (c[t] >= 0) atomicAdd(&hist[warp * nb1 + c[t]], 1u);
+  for (int w = 0; w < kLptThreads / 32; ++w) {
+    const unsigned t = sh[w];
+    if (w < warp) before += t;
+    all += t;
   }
-  // realised per-head workload
-  for (long long bh = warp; bh < BH; bh += NW) {
+  __syncthreads();   // sh may be reused by the caller
+  *total = all;
+  return before + incl - v;
+}
+
+// grid.x = (Nb + 1) + BH.  CTA c <= Nb places the items whose count is c: they start
+// after every item with a larger count (descending order) and keep their item order
+// (ties by item id ascending).  Each thread owns a contiguous run of items, counts the
+// larger and equal ones in a first pass over the counts, and after a block scan writes
+// its equal items in order in a second pass.  The remaining BH CTAs write
+// W_h = sum of the counts of head h.  No atomics: the result is deterministic.
+__global__ void __launch_bounds__(kLptThreads) lpt_kernel(const int32_t* __restrict__ counts, long long BH, int Nb,
+                                                          int64_t* __restrict__ head_work,
+                                                          int32_t* __restrict__ worklist) {
+  __shared__ unsigned sh[kLptThreads / 32];
+  __shared__ long long shs[kLptThreads / 32];
+  const long long n = BH * Nb;
+  const int c = static_cast<int>(blockIdx.x);
+  if (c > Nb) {   // realised per-head workload
+    const long long bh = c - (Nb + 1);
     long long s = 0;
-    for (int i0 = 0; i0 < Nb; i0 += 32 * kLptBatch) {
-      int c[kLptBatch];
-#pragma unroll
-      for (int t = 0; t < kLptBatch; ++t) {
-        const int i = i0 + lane + 32 * t;
-        c[t] = i < Nb ? cs[bh * Nb + i] : 0;
-      }
-#pragma unroll
-      for (int t = 0; t < kLptBatch; ++t) s += c[t];
-    }
+    for (int i = threadIdx.x; i < Nb; i += kLptThreads) s += __ldg(counts + bh * Nb + i);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if (lane == 0) head_work[bh] = s;
+    if ((threadIdx.x & 31) == 0) shs[threadIdx.x >> 5] = s;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      long long t = 0;
+      for (int w = 0; w < kLptThreads / 32; ++w) t += shs[w];
+      head_work[bh] = t;
+    }
+    return;
   }
-  __syncthreads();
-  // per count value: total over the chunks (kept in start[] for now)
-  for (int v = threadIdx.x; v < nb1; v += blockDim.x) {
-    unsigned t = 0;
-#pragma unroll
-    for (int w = 0; w < NW; ++w) t += hist[w * nb1 + v];
-    start[v] = t;
+  const long long per = (n + kLptThreads - 1) / kLptThreads;
+  const long long lo = threadIdx.x * per;
+  const long long hi = min(n, lo + per);
+  unsigned gt = 0, eq = 0;
+#pragma unroll 8
+  for (long long u = lo; u < hi; ++u) {
+    const int v = __ldg(counts + u);
+    gt += v > c ? 1u : 0u;
+    eq += v == c ? 1u : 0u;
   }
-  __syncthreads();
-  // exclusive scan over count values from high to low (warp 0; lane l owns a run)
-  if (warp == 0) {
-    const int per = (nb1 + 31) / 32;
-    unsigned tot = 0;
-    for (int q = 0; q < per; ++q) {
-      const int v = Nb - lane * per - q;
-      if (v >= 0) tot += start[v];
-    }
-    unsigned incl = tot;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    unsigned run = incl - tot;
-    for (int q = 0; q < per; ++q) {
-      const int v = Nb - lane * per - q;
-      if (v >= 0) {
-        const unsigned t = start[v];
-        start[v] = run;
-        run += t;
-      }
-    }
-  }
-  __syncthreads();
-  // per-warp cursors: warp w's items of count v follow those of warps < w
-  for (int v = threadIdx.x; v < nb1; v += blockDim.x) {
-    unsigned run = start[v];
-#pragma unroll
-    for (int w = 0; w < NW; ++w) {
-      const unsigned t = hist[w * nb1 + v];
-      hist[w * nb1 + v] = run;
-      run += t;
-    }
-  }
-  __syncthreads();
-  // stable scatter in item order within each warp's chunk, 32 items per step
-  for (long long base = lo; base < hi; base += 32 * kLptBatch) {
-    int c[kLptBatch];
-#pragma unroll
-    for (int t = 0; t < kLptBatch; ++t) {
-      const long long u = base + lane + 32 * t;
-      c[t] = u < hi ? cs[u] : -1;
-    }
-#pragma unroll
-    for (int t = 0; t < kLptBatch; ++t) {
-      const long long u = base + lane + 32 * t;
-      const bool valid = c[t] >= 0;
-      const unsigned peers = __match_any_sync(0xffffffffu, c[t]);
-      const int rank = __popc(peers & ((1u << lane) - 1u));
-      const int leader = __ffs(peers) - 1;
-      const unsigned basepos = valid ? hist[warp * nb1 + c[t]] : 0u;
-      __syncwarp();
-      if (valid && lane == leader) hist[warp * nb1 + c[t]] = basepos + __popc(peers);
-      __syncwarp();
-      if (valid) worklist[basepos + rank] = static_cast<int32_t>(u);
-    }
-  }
+  unsigned larger, equal;
+  (void)block_exclusive_scan(gt, &larger, sh);
+  unsigned pos = block_exclusive_scan(eq, &equal, sh) + larger;
+  if (equal == 0 || eq == 0) return;   // nothing of this count in this thread's run
+#pragma unroll 8
+  for (long long u = lo; u < hi; ++u)
+    if (__ldg(counts + u) == c) worklist[pos++] = static_cast<int32_t>(u);
 }
 
 }  // namespace
 
 cudaError_t launch_lpt(const int32_t* counts, const Dims& D, int64_t* head_work, int32_t* worklist, cudaStream_t s,
                        int* launches) {
-  // 32 warps with the counts staged in shared memory when everything fits, else 16
-  // warps reading the counts from global memory
-  constexpr size_t kMaxSmem = 227 * 1024;
-  const size_t nb1 = static_cast<size_t>(D.Nb) + 1;
-  const size_t n = static_cast<size_t>(D.rows());
-  const size_t big = (32 + 1) * nb1 * sizeof(unsigned) + n * sizeof(int32_t);
-  cudaError_t e;
-  if (big <= kMaxSmem) {
-    e = cudaFuncSetAttribute(lpt_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(big));
-    if (e != cudaSuccess) return e;
-    lpt_kernel<32><<<1, 32 * 32, big, s>>>(counts, D.BH(), D.Nb, 1, head_work, worklist);
-  } else {
-    const size_t small = (16 + 1) * nb1 * sizeof(unsigned);
-    e = cudaFuncSetAttribute(lpt_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(small));
-    if (e != cudaSuccess) return e;
-    lpt_kernel<16><<<1, 16 * 32, small, s>>>(counts, D.BH(), D.Nb, 0, head_work, worklist);
-  }
+  const unsigned grid = static_cast<unsigned>(D.Nb + 1 + D.BH());
+  lpt_kernel<<<grid, kLptThreads, 0, s>>>(counts, D.BH(), D.Nb, head_work, worklist);
   ++*launches;
   return cudaGetLastError();
 }
