@@ -492,7 +492,7 @@ constexpr size_t select_smem_bytes() {
 // MINB CTAs per SM; KU = unrolled k-steps of the logits loop for that register budget.
 template <int D, int PL, int R, int MINB>
 __global__ void __launch_bounds__(kRouteThreads, MINB) select_kernel(const RouteArgs a, long long bh0) {
-  constexpr int KU = MINB >= 4 ? 2 : (MINB == 3 ? 4 : 8);
+  constexpr int KU = MINB >= 4 ? 4 : (MINB == 3 ? 4 : 8);
   extern __shared__ __align__(16) unsigned char sel_smem[];
   select_item<D, PL, R, KU>(a, bh0 + blockIdx.y, static_cast<int>(blockIdx.x) * R, sel_smem);
 }
