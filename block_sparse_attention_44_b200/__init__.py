@@ -84,6 +84,8 @@ def _load():
         "fva_route": ([vp, vp, _Geom, f64, i32, vp, vp, vp, vp, sz, vp], ctypes.c_int),
         "fva_route_static": ([vp, vp, _Geom, f64, i32, vp, vp, vp, vp], ctypes.c_int),
         "fva_route_repair": ([vp, vp, _Geom, f64, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
+        "fva_reorder_pool": ([vp, vp, vp, _Geom, vp], ctypes.c_int),
+        "fva_route_repair_pooled": ([vp, vp, _Geom, f64, i32, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
         "fva_repair_workspace_size": ([_Geom], sz),
         "fva_repair": ([vp, vp, _Geom, i32, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
         "fva_block_sparse_attn": ([vp, vp, vp, vp, vp, vp, _Geom, f32, vp, vp], ctypes.c_int),
@@ -147,6 +149,15 @@ def fva_inverse_reorder(xr: torch.Tensor, x: torch.Tensor, g: Geom, stream=None)
     _check(lib.fva_inverse_reorder(_ptr(xr), _ptr(x), g.c(), _stream(stream)))
 
 
+def fva_reorder_pool(x: torch.Tensor, xr: torch.Tensor, pooled: torch.Tensor, g: Geom, stream=None) -> None:
+    """fva_reorder that also writes the float64 tile means (routing's pooled Q or K)."""
+    shp = (g.B, g.H, g.N, g.d)
+    _need(x, torch.bfloat16, shp, "x")
+    _need(xr, torch.bfloat16, shp, "xr")
+    _need(pooled, torch.float64, (g.B, g.H, g.Nb, g.d), "pooled")
+    _check(lib.fva_reorder_pool(_ptr(x), _ptr(xr), _ptr(pooled), g.c(), _stream(stream)))
+
+
 def fva_route_workspace_size(g: Geom) -> int:
     return int(lib.fva_route_workspace_size(g.c()))
 
@@ -202,6 +213,24 @@ def fva_route_repair(qr, kr, g: Geom, p: float, k: int, counts, idx, head_work, 
     _check(lib.fva_route_repair(_ptr(qr), _ptr(kr), g.c(), float(p), int(k), _ptr(topp_mask), _ptr(topk_idx),
                                 _ptr(counts), _ptr(idx), _ptr(head_work), _ptr(worklist), _ptr(workspace),
                                 workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def fva_route_repair_pooled(qbar, kbar, g: Geom, p: float, k: int, counts, idx, head_work, worklist,
+                            topp_mask=None, topk_idx=None, stream=None):
+    """fva_route_repair from block means already computed (fva_reorder_pool)."""
+    _need(qbar, torch.float64, (g.B, g.H, g.Nb, g.d), "qbar")
+    _need(kbar, torch.float64, (g.B, g.H, g.Nb, g.d), "kbar")
+    if topp_mask is not None:
+        _need(topp_mask, torch.uint8, (g.B, g.H, g.Nb, g.Nb), "topp_mask")
+    if topk_idx is not None:
+        _need(topk_idx, torch.int32, (g.B, g.H, g.Nb, min(k, g.Nb)), "topk_idx")
+    _need(counts, torch.int32, (g.B, g.H, g.Nb), "counts")
+    _need(idx, torch.int32, (g.B, g.H, g.Nb, g.Nb), "idx")
+    _need(head_work, torch.int64, (g.B, g.H), "head_work")
+    _need(worklist, torch.int32, (g.B * g.H * g.Nb,), "worklist")
+    _check(lib.fva_route_repair_pooled(_ptr(qbar), _ptr(kbar), g.c(), float(p), int(k), _ptr(topp_mask),
+                                       _ptr(topk_idx), _ptr(counts), _ptr(idx), _ptr(head_work), _ptr(worklist),
+                                       _stream(stream)))
 
 
 def fva_repair_workspace_size(g: Geom) -> int:
@@ -274,8 +303,9 @@ class SparseAttention:
 
     Buffers are allocated once through PyTorch for a geometry; `__call__` only
     enqueues library kernels on the current (or given) stream.  With fused=True
-    (default) routing and repair run as fva_route_repair and the Top-p mask / Top-k
-    ids are not materialised; fused=False runs fva_route then fva_repair.
+    (default) Q and K are pooled by their reorder pass (fva_reorder_pool), routing and
+    repair run as fva_route_repair_pooled and the Top-p mask / Top-k ids are not
+    materialised; fused=False runs fva_reorder, fva_route, then fva_repair.
     """
 
     def __init__(self, g: Geom, p: float, k: int, device="cuda", use_lpt: bool = True,
@@ -293,12 +323,14 @@ class SparseAttention:
                                  torch.empty((g.B, g.H), dtype=torch.int64, device=dev),
                                  torch.empty((g.B * g.H * g.Nb,), dtype=torch.int32, device=dev))
         self.ws = torch.empty((max(fva_route_workspace_size(g), 256),), dtype=torch.uint8, device=dev)
+        self.qbar, self.kbar = (torch.empty((g.B, g.H, g.Nb, g.d), dtype=torch.float64, device=dev)
+                                for _ in range(2))
 
     def routing(self, stream=None) -> None:
         g = self.g
-        if self.fused:
-            fva_route_repair(self.qr, self.kr, g, self.p, self.k, self.rep.counts, self.rep.idx, self.rep.head_work,
-                             self.rep.worklist, self.ws, stream=stream)
+        if self.fused:   # the means come from the reorder pass (reorder_qk)
+            fva_route_repair_pooled(self.qbar, self.kbar, g, self.p, self.k, self.rep.counts, self.rep.idx,
+                                    self.rep.head_work, self.rep.worklist, stream=stream)
             return
         fva_route(self.qr, self.kr, g, self.p, self.k, self.route.topp_mask, self.route.topk_idx, self.ws,
                   stream=stream)
@@ -310,11 +342,19 @@ class SparseAttention:
                               self.rep.worklist if self.use_lpt else None, self.g, self.scale, self.outr,
                               stream=stream)
 
+    def reorder_qkv(self, q, k, v, stream=None) -> None:
+        g = self.g
+        if self.fused:
+            fva_reorder_pool(q, self.qr, self.qbar, g, stream)
+            fva_reorder_pool(k, self.kr, self.kbar, g, stream)
+        else:
+            fva_reorder(q, self.qr, g, stream)
+            fva_reorder(k, self.kr, g, stream)
+        fva_reorder(v, self.vr, g, stream)
+
     def __call__(self, q, k, v, out, stream=None) -> torch.Tensor:
         g = self.g
-        fva_reorder(q, self.qr, g, stream)
-        fva_reorder(k, self.kr, g, stream)
-        fva_reorder(v, self.vr, g, stream)
+        self.reorder_qkv(q, k, v, stream)
         self.routing(stream)
         self.attention(stream)
         fva_inverse_reorder(self.outr, out, g, stream)

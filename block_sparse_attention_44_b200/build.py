@@ -1,4 +1,5 @@
-"""Builds libfva.so (sm_100a) in-tree with nvcc.  `python -m block_sparse_attention_44_b200.build`."""
+"""Builds libfva.so (sm_100a) in-tree with nvcc.  `python block_sparse_attention_44_b200/build.py`
+(run as a script: importing the package would load the library being rebuilt)."""
 from __future__ import annotations
 
 import os

@@ -82,7 +82,7 @@ int finish(cudaError_t e, int launches, const char* where) {
 
 extern "C" {
 
-int32_t fva_version(void) { return 101; }
+int32_t fva_version(void) { return 102; }
 
 const char* fva_last_error(void) { return g_err; }
 
@@ -104,6 +104,19 @@ int fva_reorder(const void* x, void* xr, fva_geom g, void* stream) { return reor
 
 int fva_inverse_reorder(const void* xr, void* x, fva_geom g, void* stream) {
   return reorder_common(xr, x, g, stream, true);
+}
+
+int fva_reorder_pool(const void* x, void* xr, double* pooled, fva_geom g, void* stream) {
+  fva::Dims D;
+  int rc = check_geom(g, D, false);
+  if (rc) return rc;
+  if (!x || !xr || !pooled) return fail(FVA_ERR_INVALID_ARG, "null pointer");
+  if (x == xr) return fail(FVA_ERR_INVALID_ARG, "in-place reorder is not supported");
+  if (!aligned16(x) || !aligned16(xr)) return fail(FVA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(pooled) & 7u) != 0) return fail(FVA_ERR_INVALID_ARG, "pooled must be 8-byte aligned");
+  int launches = 0;
+  cudaError_t e = fva::launch_reorder_pool(x, xr, pooled, g, D, static_cast<cudaStream_t>(stream), &launches);
+  return finish(e, launches, "fva_reorder_pool");
 }
 
 size_t fva_route_workspace_size(fva_geom g) {
@@ -158,6 +171,26 @@ int fva_route_repair(const void* qr, const void* kr, fva_geom g, double p, int32
                                     &launches);
   if (e == cudaSuccess) e = fva::launch_lpt(counts, D, head_work, worklist, s, &launches);
   return finish(e, launches, "fva_route_repair");
+}
+
+int fva_route_repair_pooled(const double* qbar, const double* kbar, fva_geom g, double p, int32_t k,
+                            uint8_t* topp_mask, int32_t* topk_idx, int32_t* counts, int32_t* idx,
+                            int64_t* head_work, int32_t* worklist, void* stream) {
+  fva::Dims D;
+  int rc = check_geom(g, D, false);
+  if (rc) return rc;
+  if (!qbar || !kbar || !counts || !idx || !head_work || !worklist) return fail(FVA_ERR_INVALID_ARG, "null pointer");
+  if (!(p > 0.0) || !(p <= 1.0)) return fail(FVA_ERR_INVALID_ARG, "p must satisfy 0 < p <= 1 (got %g)", p);
+  if (k < 1) return fail(FVA_ERR_INVALID_ARG, "k must be >= 1 (got %d)", k);
+  if (D.Nb > fva::kMaxNb) return fail(FVA_ERR_UNSUPPORTED, "Nb = %d blocks exceeds %d", D.Nb, fva::kMaxNb);
+  if (!aligned16(qbar) || !aligned16(kbar)) return fail(FVA_ERR_INVALID_ARG, "qbar and kbar must be 16-byte aligned");
+  const int kk = k < D.Nb ? k : D.Nb;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int launches = 0;
+  cudaError_t e = fva::launch_select_pooled(qbar, kbar, D, p, kk, topp_mask, topk_idx, nullptr, counts, idx, s,
+                                            &launches);
+  if (e == cudaSuccess) e = fva::launch_lpt(counts, D, head_work, worklist, s, &launches);
+  return finish(e, launches, "fva_route_repair_pooled");
 }
 
 size_t fva_repair_workspace_size(fva_geom g) {

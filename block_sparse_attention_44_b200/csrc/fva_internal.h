@@ -21,6 +21,10 @@ constexpr int kMaxNb = 2048;
 cudaError_t launch_reorder(const void* src, void* dst, const fva_geom& g, const Dims& D, bool inverse,
                            cudaStream_t s, int* launches);
 
+// Forward reorder that also writes the float64 mean of every tile ([B*H*Nb, d]).
+cudaError_t launch_reorder_pool(const void* src, void* dst, double* pooled, const fva_geom& g, const Dims& D,
+                                cudaStream_t s, int* launches);
+
 // Routing: block means (float64), float64 logits, Top-p / Top-k selection; with
 // counts != nullptr also the repaired, compacted per-row lists (idx, counts).
 // topp_mask, topk_idx and logits_out may each be null (not written).
@@ -28,6 +32,11 @@ cudaError_t launch_route(const void* qr, const void* kr, const Dims& D, double p
                          int32_t* topk_idx, double* logits_out, int32_t* counts, int32_t* idx, void* ws,
                          cudaStream_t s, int* launches);
 size_t route_workspace_bytes(const Dims& D);
+// Scoring and selection (and compaction when counts != nullptr) from block means the
+// caller already holds (e.g. written by launch_reorder_pool).
+cudaError_t launch_select_pooled(const double* qbar, const double* kbar, const Dims& D, double p, int kk,
+                                 uint8_t* topp_mask, int32_t* topk_idx, double* logits_out, int32_t* counts,
+                                 int32_t* idx, cudaStream_t s, int* launches);
 
 // Repair + compaction + per-head work + LPT work list.
 cudaError_t launch_repair(const uint8_t* topp_mask, const int32_t* topk_idx, const Dims& D, int kk, int32_t* counts,

@@ -536,13 +536,12 @@ size_t route_workspace_bytes(const Dims& D) {
   return 2 * align_up(pooled);
 }
 
-cudaError_t launch_route(const void* qr, const void* kr, const Dims& D, double p, int kk, uint8_t* topp_mask,
-                         int32_t* topk_idx, double* logits_out, int32_t* counts, int32_t* idx, void* ws,
-                         cudaStream_t s, int* launches) {
-  const Carve c = carve(D, ws);
+namespace {
+RouteArgs make_args(const double* qbar, const double* kbar, const Dims& D, double p, int kk, uint8_t* topp_mask,
+                    int32_t* topk_idx, double* logits_out, int32_t* counts, int32_t* idx) {
   RouteArgs a;
-  a.qbar = c.qbar;
-  a.kbar = c.kbar;
+  a.qbar = qbar;
+  a.kbar = kbar;
   a.topp_mask = topp_mask;
   a.topk_idx = topk_idx;
   a.logits_out = logits_out;
@@ -553,7 +552,24 @@ cudaError_t launch_route(const void* qr, const void* kr, const Dims& D, double p
   a.keep_all_p = p >= 1.0 ? 1 : 0;
   const double tp = ceil(p * 0x1p31);
   a.target = a.keep_all_p ? 0u : static_cast<unsigned>(tp < 1.0 ? 1.0 : tp);
+  return a;
+}
+}  // namespace
 
+cudaError_t launch_select_pooled(const double* qbar, const double* kbar, const Dims& D, double p, int kk,
+                                 uint8_t* topp_mask, int32_t* topk_idx, double* logits_out, int32_t* counts,
+                                 int32_t* idx, cudaStream_t s, int* launches) {
+  const RouteArgs a = make_args(qbar, kbar, D, p, kk, topp_mask, topk_idx, logits_out, counts, idx);
+  cudaError_t e = D.d == 128 ? launch_select<128>(a, 0, D.BH(), s) : launch_select<64>(a, 0, D.BH(), s);
+  ++*launches;
+  return e;
+}
+
+cudaError_t launch_route(const void* qr, const void* kr, const Dims& D, double p, int kk, uint8_t* topp_mask,
+                         int32_t* topk_idx, double* logits_out, int32_t* counts, int32_t* idx, void* ws,
+                         cudaStream_t s, int* launches) {
+  const Carve c = carve(D, ws);
+  const RouteArgs a = make_args(c.qbar, c.kbar, D, p, kk, topp_mask, topk_idx, logits_out, counts, idx);
   const long long rows = D.rows();
   const dim3 pgrid(static_cast<unsigned>(2 * rows));
   if (D.d == 128)

@@ -10,6 +10,8 @@
  *   fva_repair           forced diagonal + floor, compaction into per-row key-block lists,
  *                        per-head realised workload, heavy-first (LPT) work list
  *   fva_route_repair     the two above, fused
+ *   fva_reorder_pool, fva_route_repair_pooled
+ *                        the same with the pooling done by the reorder pass
  *   fva_block_sparse_attn  flash-style attention over the kept block pairs
  *   fva_inverse_reorder  back to natural token order
  *
@@ -66,6 +68,18 @@ int fva_reorder(const void* x, void* xr, fva_geom g, void* stream);
  * token order on the output; §3.1 overview, final stage).  Same constraints.
  */
 int fva_inverse_reorder(const void* xr, void* x, fva_geom g, void* stream);
+
+/*
+ * fva_reorder_pool — fva_reorder that also writes the routing block means (the pooled
+ * Q or K of §3.1) while the tile passes through: the pooling step costs no second read
+ * of the tensor.
+ *   x, xr  : as in fva_reorder.
+ *   pooled : float64 [B,H,Nb,d] output, pooled[b,h,i,:] = mean of the S rows of tile i
+ *            (8-byte aligned; 16-byte aligned if it feeds fva_route_repair_pooled).
+ * The means are summed in the same order as fva_route's own pooling, so they are
+ * bit-identical to what fva_route computes internally.
+ */
+int fva_reorder_pool(const void* x, void* xr, double* pooled, fva_geom g, void* stream);
 
 /* Workspace bytes fva_route needs for geometry g (pooled Q and K, float64). */
 size_t fva_route_workspace_size(fva_geom g);
@@ -135,6 +149,16 @@ int fva_route_repair(const void* qr, const void* kr, fva_geom g, double p, int32
                      uint8_t* topp_mask, int32_t* topk_idx, int32_t* counts, int32_t* idx,
                      int64_t* head_work, int32_t* worklist,
                      void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * fva_route_repair_pooled — fva_route_repair from block means the caller already holds
+ * (fva_reorder_pool outputs for Q and K): scoring, Top-p / Top-k selection, repair,
+ * W_h and the LPT list, with the same outputs and arithmetic.  No workspace.
+ *   qbar, kbar : float64 [B,H,Nb,d], 16-byte aligned.
+ */
+int fva_route_repair_pooled(const double* qbar, const double* kbar, fva_geom g, double p, int32_t k,
+                            uint8_t* topp_mask, int32_t* topk_idx, int32_t* counts, int32_t* idx,
+                            int64_t* head_work, int32_t* worklist, void* stream);
 
 /* Workspace bytes fva_repair needs (currently 0; kept for ABI stability). */
 size_t fva_repair_workspace_size(fva_geom g);

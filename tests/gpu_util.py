@@ -58,8 +58,20 @@ def run_path(fva, g, q, k, v, p, kfloor, use_lpt=True, want_logits=False):
     fva.fva_inverse_reorder(outr, out, g)
     torch.cuda.synchronize()
     assert fva.fva_get_device_error() == 0
+    # pooling done by the reorder pass, then routing from those means
+    qbar, kbar = (torch.empty((g.B, g.H, g.Nb, g.d), dtype=torch.float64, device="cuda") for _ in range(2))
+    qr2, kr2 = torch.empty_like(qr), torch.empty_like(kr)
+    fva.fva_reorder_pool(qd, qr2, qbar, g)
+    fva.fva_reorder_pool(kd, kr2, kbar, g)
+    pooled = dict(counts=torch.empty_like(counts), idx=torch.full_like(idx, -1), head_work=torch.empty_like(hw),
+                  worklist=torch.empty_like(wl), mask=torch.empty_like(mask), topk=torch.empty_like(topk))
+    fva.fva_route_repair_pooled(qbar, kbar, g, p, kfloor, pooled["counts"], pooled["idx"], pooled["head_work"],
+                                pooled["worklist"], topp_mask=pooled["mask"], topk_idx=pooled["topk"])
+    torch.cuda.synchronize()
+    assert fva.fva_get_device_error() == 0
     dev.update(qr=qr, kr=kr, vr=vr, mask=mask, topk=topk, logits=logits, counts=counts, idx=idx, head_work=hw,
-               worklist=wl, outr=outr, out=out, fused=fused, bare=bare)
+               worklist=wl, outr=outr, out=out, fused=fused, bare=bare, pooled=pooled, qr2=qr2, kr2=kr2, qbar=qbar,
+               kbar=kbar)
     return dev
 
 
@@ -73,6 +85,22 @@ def check_fused(dev: dict):
         assert torch.equal(torch.where(valid, res["idx"], -1), torch.where(valid, dev["idx"], -1))
     assert torch.equal(dev["fused"]["mask"], dev["mask"])
     assert torch.equal(dev["fused"]["topk"], dev["topk"])
+
+
+def check_pooled(dev: dict, q: np.ndarray, k: np.ndarray, og):
+    """fva_reorder_pool reorders exactly like fva_reorder and its means match the oracle's
+    pooling; routing from those means gives exactly the lists of the other entry points."""
+    assert torch.equal(dev["qr2"].view(torch.int16), dev["qr"].view(torch.int16))
+    assert torch.equal(dev["kr2"].view(torch.int16), dev["kr"].view(torch.int16))
+    for bar, x in ((dev["qbar"], q), (dev["kbar"], k)):
+        want = O.pool_blocks(O.reorder(x, og), og.S)
+        assert np.allclose(bar.cpu().numpy(), want, rtol=1e-13, atol=1e-15)
+    res = dev["pooled"]
+    for key in ("counts", "head_work", "worklist", "mask", "topk"):
+        assert torch.equal(res[key], dev[key]), key
+    Nb = dev["idx"].shape[-1]
+    valid = torch.arange(Nb, device=dev["idx"].device)[None, None, None, :] < dev["counts"][..., None]
+    assert torch.equal(torch.where(valid, res["idx"], -1), torch.where(valid, dev["idx"], -1))
 
 
 def check_route(rr: O.RouteResult, mask_dev: np.ndarray, topk_dev: np.ndarray, max_tie_frac=0.02):

@@ -88,6 +88,18 @@ def test_invalid_arguments_rejected_on_host():
     assert L.fva_route_repair(256, 512, g, 0.9, 1, None, None, None, 32, 64, 128, 4096, need, None) == \
         fva.FVA_ERR_INVALID_ARG
     assert b"null" in L.fva_last_error()
+    # reorder with pooling, routing from pooled means
+    assert L.fva_reorder_pool(16, 32, None, g, None) == fva.FVA_ERR_INVALID_ARG
+    assert L.fva_reorder_pool(16, 16, 64, g, None) == fva.FVA_ERR_INVALID_ARG            # in place
+    assert L.fva_reorder_pool(16, 32, 68, g, None) == fva.FVA_ERR_INVALID_ARG            # pooled misaligned
+    assert L.fva_reorder_pool(16, 32, 64, bad, None) == fva.FVA_ERR_INVALID_ARG
+    pargs = lambda p, k: (256, 512, g, p, k, None, None, 16, 32, 64, 128, None)
+    assert L.fva_route_repair_pooled(*pargs(0.0, 1)) == fva.FVA_ERR_INVALID_ARG
+    assert L.fva_route_repair_pooled(*pargs(0.9, 0)) == fva.FVA_ERR_INVALID_ARG
+    assert L.fva_route_repair_pooled(None, 512, g, 0.9, 1, None, None, 16, 32, 64, 128, None) == \
+        fva.FVA_ERR_INVALID_ARG
+    assert L.fva_route_repair_pooled(264, 512, g, 0.9, 1, None, None, 16, 32, 64, 128, None) == \
+        fva.FVA_ERR_INVALID_ARG                                                           # qbar misaligned
     # repair / attention: null pointers, k, unsupported tile for attention
     assert L.fva_repair(None, 16, g, 1, 16, 16, 16, 16, None, 0, None) == fva.FVA_ERR_INVALID_ARG
     assert L.fva_repair(16, 16, g, 0, 16, 16, 16, 16, None, 0, None) == fva.FVA_ERR_INVALID_ARG

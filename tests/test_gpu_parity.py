@@ -13,8 +13,8 @@ pytestmark = pytest.mark.gpu
 
 import oracle as O
 import synth
-from gpu_util import (bf16_dev_to_f64, check_fused, check_repair, check_route, compare_attention, run_path, to_bits,
-                      to_dev)
+from gpu_util import (bf16_dev_to_f64, check_fused, check_pooled, check_repair, check_route, compare_attention, run_path,
+                      to_bits, to_dev)
 
 
 @pytest.fixture(scope="module")
@@ -75,6 +75,7 @@ def test_path_matches_oracle(fva, name):
     rp = check_repair(dev, mask_dev, topk_dev)
     assert (rp.counts >= min(cfg.k, og.Nb)).all()
     check_fused(dev)
+    check_pooled(dev, q, k, og)
 
     # a6: attention with the device index lists, all items
     want = O.attention(qr, kr, vr, rp.counts, rp.idx, og.S)
