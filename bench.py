@@ -268,7 +268,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
     # --- timed region: K whole steps; per-stage events on the launching stream
     K = args.steps
     E = lambda: torch.cuda.Event(enable_timing=True)
-    ev = [[E() for _ in range(5)] for _ in range(K)]
+    ev = [[E() for _ in range(4)] for _ in range(K)]
     gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
     if world > 1:
         dist.barrier()
@@ -284,10 +284,8 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
             e[1].record(stream)
             path.routing(stream)                  # fva_route_repair_pooled: select + repair + LPT list
             e[2].record(stream)
-            path.attention(stream)
+            path.attention_natural(out, stream)   # attention, output written in natural order
             e[3].record(stream)
-            fva.fva_inverse_reorder(path.outr, out, g, stream)
-            e[4].record(stream)
         stop.record(stream)
         torch.cuda.synchronize(dev)
     launches = fva.fva_launch_count() - launches0
@@ -298,8 +296,8 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         total_ms = float(t.item())
     ms = total_ms / K
-    stage = np.array([[ev[s][i].elapsed_time(ev[s][i + 1]) for i in range(4)] for s in range(K)])
-    st_mean = stage.mean(axis=0)            # reorder x3, route + repair (fused), attention, inverse (ms)
+    stage = np.array([[ev[s][i].elapsed_time(ev[s][i + 1]) for i in range(3)] for s in range(K)])
+    st_mean = stage.mean(axis=0)            # reorder x3 (+ pooling), routing from the means, attention (ms)
     attn_ms = float(st_mean[2])
     route_ms = float(st_mean[1])
 
@@ -373,8 +371,8 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
                                     / 1e9 / peaks["hbm_gbs"],
         "reorder_gbs": bytes_reorder / (st_mean[0] * 1e-3) / 1e9,
         "routing_overhead_pct": 100.0 * route_ms / attn_ms,
-        "stage_ms": {"reorder_qkv_pool": st_mean[0], "route_repair_from_pooled": st_mean[1], "attention": st_mean[2],
-                     "inverse_reorder": st_mean[3], "route_repair_fused": fused_route_ms,
+        "stage_ms": {"reorder_qkv_pool": st_mean[0], "route_repair_from_pooled": st_mean[1],
+                     "attention_natural_out": st_mean[2], "route_repair_fused": fused_route_ms,
                      "route_unfused": sep_route_ms, "repair_unfused": sep_repair_ms},
         "routing_unfused_gbs": bytes_route / ((sep_route_ms + sep_repair_ms) * 1e-3) / 1e9,
         "roofline": {"bound": "tensor", "kernel": "attn_kernel (fva_block_sparse_attn)", "achieved": achieved,

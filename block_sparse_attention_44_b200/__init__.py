@@ -89,6 +89,7 @@ def _load():
         "fva_repair_workspace_size": ([_Geom], sz),
         "fva_repair": ([vp, vp, _Geom, i32, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
         "fva_block_sparse_attn": ([vp, vp, vp, vp, vp, vp, _Geom, f32, vp, vp], ctypes.c_int),
+        "fva_block_sparse_attn_natural": ([vp, vp, vp, vp, vp, vp, _Geom, f32, vp, vp], ctypes.c_int),
         "fva_get_device_error": ([vp, ctypes.POINTER(i32)], ctypes.c_int),
         "fva_last_error": ([], ctypes.c_char_p),
         "fva_launch_count": ([], i64),
@@ -261,6 +262,20 @@ def fva_block_sparse_attn(qr, kr, vr, counts, idx, worklist, g: Geom, softmax_sc
                                      float(softmax_scale), _ptr(out_r), _stream(stream)))
 
 
+def fva_block_sparse_attn_natural(qr, kr, vr, counts, idx, worklist, g: Geom, softmax_scale: float, out,
+                                  stream=None):
+    """fva_block_sparse_attn writing the output in natural token order (inverse reorder fused)."""
+    shp = (g.B, g.H, g.N, g.d)
+    for t, n in ((qr, "qr"), (kr, "kr"), (vr, "vr"), (out, "out")):
+        _need(t, torch.bfloat16, shp, n)
+    _need(counts, torch.int32, (g.B, g.H, g.Nb), "counts")
+    _need(idx, torch.int32, (g.B, g.H, g.Nb, g.Nb), "idx")
+    if worklist is not None:
+        _need(worklist, torch.int32, (g.B * g.H * g.Nb,), "worklist")
+    _check(lib.fva_block_sparse_attn_natural(_ptr(qr), _ptr(kr), _ptr(vr), _ptr(counts), _ptr(idx), _ptr(worklist),
+                                             g.c(), float(softmax_scale), _ptr(out), _stream(stream)))
+
+
 def fva_get_device_error(stream=None) -> int:
     """Synchronises the stream; returns (and clears) the device error word, 0 if none."""
     code = ctypes.c_int32(0)
@@ -338,9 +353,16 @@ class SparseAttention:
                    self.rep.head_work, self.rep.worklist, stream=stream)
 
     def attention(self, stream=None) -> None:
+        """Tile-major output into self.outr."""
         fva_block_sparse_attn(self.qr, self.kr, self.vr, self.rep.counts, self.rep.idx,
                               self.rep.worklist if self.use_lpt else None, self.g, self.scale, self.outr,
                               stream=stream)
+
+    def attention_natural(self, out, stream=None) -> None:
+        """Natural-order output into `out` (the inverse reorder fused into the epilogue)."""
+        fva_block_sparse_attn_natural(self.qr, self.kr, self.vr, self.rep.counts, self.rep.idx,
+                                      self.rep.worklist if self.use_lpt else None, self.g, self.scale, out,
+                                      stream=stream)
 
     def reorder_qkv(self, q, k, v, stream=None) -> None:
         g = self.g
@@ -356,6 +378,9 @@ class SparseAttention:
         g = self.g
         self.reorder_qkv(q, k, v, stream)
         self.routing(stream)
-        self.attention(stream)
-        fva_inverse_reorder(self.outr, out, g, stream)
+        if self.fused:
+            self.attention_natural(out, stream)
+        else:
+            self.attention(stream)
+            fva_inverse_reorder(self.outr, out, g, stream)
         return out

@@ -87,7 +87,26 @@ struct AttnParams {
   int N;
   int Nb;
   float scale_log2;
+  // natural != 0: row r of tile i is written at its natural token position (the inverse
+  // reorder fused into the epilogue); grid X, Y and tile tt x ty x tx, nY x nX tiles
+  int natural, Y, X, tt, ty, tx, nY, nX;
 };
+
+// Token position of row r of tile i in the output: tile-major i*S + r, or the natural
+// raster index of that token when prm.natural is set.
+__device__ __forceinline__ long long out_token(const AttnParams& prm, int i, int r, int S) {
+  if (!prm.natural) return static_cast<long long>(i) * S + r;
+  const int bt = i / (prm.nY * prm.nX);
+  const int rem = i - bt * prm.nY * prm.nX;
+  const int by = rem / prm.nX;
+  const int bx = rem - by * prm.nX;
+  const int tyx = prm.ty * prm.tx;
+  const int lt = r / tyx;
+  const int rr = r - lt * tyx;
+  const int ly = rr / prm.tx;
+  const int lx = rr - ly * prm.tx;
+  return (static_cast<long long>(bt * prm.tt + lt) * prm.Y + by * prm.ty + ly) * prm.X + bx * prm.tx + lx;
+}
 
 // Work item at list position `it`; -1 (and the device error word set) if the list
 // holds an id outside [0, n_items).  Every role calls this on the same data, so all
@@ -389,7 +408,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int n = item_count(prm, item);
       const long long bh = item / Nb;
       const int i = item - static_cast<int>(bh * Nb);
-      uint16_t* orow = prm.out + (bh * prm.N + static_cast<long long>(i) * S + row) * D + half * HD;
+      uint16_t* orow = prm.out + (bh * prm.N + out_token(prm, i, row < S ? row : 0, S)) * D + half * HD;
       if (n <= 0) {
         if (row < S)
           for (int c = 0; c < HD; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
@@ -582,8 +601,8 @@ cudaError_t launch_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
 }  // namespace
 
 cudaError_t launch_attention(const void* qr, const void* kr, const void* vr, const int32_t* counts, const int32_t* idx,
-                             const int32_t* worklist, const Dims& D, float scale, void* out, int* dev_err,
-                             cudaStream_t s, int* launches, char* msg, size_t msg_len) {
+                             const int32_t* worklist, const Dims& D, const fva_geom* natural, float scale, void* out,
+                             int* dev_err, cudaStream_t s, int* launches, char* msg, size_t msg_len) {
   const long long rows = D.BH() * D.N;
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, qr, rows, D.d, D.S, msg, msg_len) || !make_map(&mk, kr, rows, D.d, D.S, msg, msg_len) ||
@@ -599,6 +618,14 @@ cudaError_t launch_attention(const void* qr, const void* kr, const void* vr, con
   prm.N = D.N;
   prm.Nb = D.Nb;
   prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.natural = natural ? 1 : 0;
+  prm.Y = natural ? natural->Y : 0;
+  prm.X = natural ? natural->X : 0;
+  prm.tt = natural ? natural->tt : 0;
+  prm.ty = natural ? natural->ty : 0;
+  prm.tx = natural ? natural->tx : 0;
+  prm.nY = D.nY;
+  prm.nX = D.nX;
   cudaError_t e;
   if (D.d == 128 && D.S == 128)
     e = launch_t<128, 128, 3, 3>(mq, mk, mv, prm, s);

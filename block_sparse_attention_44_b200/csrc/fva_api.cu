@@ -82,7 +82,7 @@ int finish(cudaError_t e, int launches, const char* where) {
 
 extern "C" {
 
-int32_t fva_version(void) { return 102; }
+int32_t fva_version(void) { return 103; }
 
 const char* fva_last_error(void) { return g_err; }
 
@@ -218,27 +218,41 @@ int fva_repair(const uint8_t* topp_mask, const int32_t* topk_idx, fva_geom g, in
   return finish(e, launches, "fva_repair");
 }
 
-int fva_block_sparse_attn(const void* qr, const void* kr, const void* vr, const int32_t* counts, const int32_t* idx,
-                          const int32_t* worklist, fva_geom g, float softmax_scale, void* out_r, void* stream) {
+static int attn_common(const void* qr, const void* kr, const void* vr, const int32_t* counts, const int32_t* idx,
+                       const int32_t* worklist, fva_geom g, float softmax_scale, void* out, void* stream,
+                       bool natural, const char* name) {
   fva::Dims D;
   int rc = check_geom(g, D, true);
   if (rc) return rc;
-  if (!qr || !kr || !vr || !counts || !idx || !out_r) return fail(FVA_ERR_INVALID_ARG, "null pointer");
-  if (!aligned16(qr) || !aligned16(kr) || !aligned16(vr) || !aligned16(out_r))
+  if (!qr || !kr || !vr || !counts || !idx || !out) return fail(FVA_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(qr) || !aligned16(kr) || !aligned16(vr) || !aligned16(out))
     return fail(FVA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
   if (!isfinite(softmax_scale)) return fail(FVA_ERR_INVALID_ARG, "softmax_scale must be finite");
   const float scale = softmax_scale > 0.0f ? softmax_scale : 1.0f / sqrtf(static_cast<float>(D.d));
   int* de = dev_err_ptr();
-  if (!de) return fail(FVA_ERR_CUDA, "fva_block_sparse_attn: cannot resolve the device error word");
+  if (!de) return fail(FVA_ERR_CUDA, "%s: cannot resolve the device error word", name);
   char msg[256] = "";
   int launches = 0;
-  cudaError_t e = fva::launch_attention(qr, kr, vr, counts, idx, worklist, D, scale, out_r, de,
+  cudaError_t e = fva::launch_attention(qr, kr, vr, counts, idx, worklist, D, natural ? &g : nullptr, scale, out, de,
                                         static_cast<cudaStream_t>(stream), &launches, msg, sizeof(msg));
   if (msg[0]) {
     g_launches += launches;
-    return fail(FVA_ERR_CUDA, "fva_block_sparse_attn: %s", msg);
+    return fail(FVA_ERR_CUDA, "%s: %s", name, msg);
   }
-  return finish(e, launches, "fva_block_sparse_attn");
+  return finish(e, launches, name);
+}
+
+int fva_block_sparse_attn(const void* qr, const void* kr, const void* vr, const int32_t* counts, const int32_t* idx,
+                          const int32_t* worklist, fva_geom g, float softmax_scale, void* out_r, void* stream) {
+  return attn_common(qr, kr, vr, counts, idx, worklist, g, softmax_scale, out_r, stream, false,
+                     "fva_block_sparse_attn");
+}
+
+int fva_block_sparse_attn_natural(const void* qr, const void* kr, const void* vr, const int32_t* counts,
+                                  const int32_t* idx, const int32_t* worklist, fva_geom g, float softmax_scale,
+                                  void* out, void* stream) {
+  return attn_common(qr, kr, vr, counts, idx, worklist, g, softmax_scale, out, stream, true,
+                     "fva_block_sparse_attn_natural");
 }
 
 int fva_get_device_error(void* stream, int32_t* code) {

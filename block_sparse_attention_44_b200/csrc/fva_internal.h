@@ -48,8 +48,9 @@ cudaError_t launch_lpt(const int32_t* counts, const Dims& D, int64_t* head_work,
                        int* launches);
 
 // Block-sparse attention (tcgen05).
+// natural != nullptr: O is written in natural token order of that geometry.
 cudaError_t launch_attention(const void* qr, const void* kr, const void* vr, const int32_t* counts, const int32_t* idx,
-                             const int32_t* worklist, const Dims& D, float scale, void* out, int* dev_err,
-                             cudaStream_t s, int* launches, char* msg, size_t msg_len);
+                             const int32_t* worklist, const Dims& D, const fva_geom* natural, float scale, void* out,
+                             int* dev_err, cudaStream_t s, int* launches, char* msg, size_t msg_len);
 
 }  // namespace fva

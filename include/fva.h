@@ -14,6 +14,7 @@
  *                        the same with the pooling done by the reorder pass
  *   fva_block_sparse_attn  flash-style attention over the kept block pairs
  *   fva_inverse_reorder  back to natural token order
+ *   fva_block_sparse_attn_natural  attention with the inverse reorder fused
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -195,6 +196,17 @@ int fva_repair(const uint8_t* topp_mask, const int32_t* topk_idx, fva_geom g, in
 int fva_block_sparse_attn(const void* qr, const void* kr, const void* vr,
                           const int32_t* counts, const int32_t* idx, const int32_t* worklist,
                           fva_geom g, float softmax_scale, void* out_r, void* stream);
+
+/*
+ * fva_block_sparse_attn_natural — fva_block_sparse_attn writing O in natural token
+ * order: the inverse reorder (§3.1, final stage) fused into the epilogue, so the
+ * output is written once and not permuted in a second pass.  Same arguments; `out` is
+ * bf16 [B,H,N,d] in natural order (bit-identical to fva_inverse_reorder of the
+ * tile-major result).
+ */
+int fva_block_sparse_attn_natural(const void* qr, const void* kr, const void* vr,
+                                  const int32_t* counts, const int32_t* idx, const int32_t* worklist,
+                                  fva_geom g, float softmax_scale, void* out, void* stream);
 
 /*
  * fva_get_device_error — synchronises `stream`, then reads and clears the device

@@ -56,8 +56,12 @@ def run_path(fva, g, q, k, v, p, kfloor, use_lpt=True, want_logits=False):
                          ws)
     fva.fva_block_sparse_attn(qr, kr, vr, counts, idx, wl if use_lpt else None, g, 0.0, outr)
     fva.fva_inverse_reorder(outr, out, g)
+    out_nat = torch.empty_like(out)
+    fva.fva_block_sparse_attn_natural(qr, kr, vr, counts, idx, wl if use_lpt else None, g, 0.0, out_nat)
     torch.cuda.synchronize()
     assert fva.fva_get_device_error() == 0
+    # the fused epilogue writes exactly the inverse reorder of the tile-major output
+    assert torch.equal(out_nat.view(torch.int16), out.view(torch.int16))
     # pooling done by the reorder pass, then routing from those means
     qbar, kbar = (torch.empty((g.B, g.H, g.Nb, g.d), dtype=torch.float64, device="cuda") for _ in range(2))
     qr2, kr2 = torch.empty_like(qr), torch.empty_like(kr)

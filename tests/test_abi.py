@@ -104,6 +104,9 @@ def test_invalid_arguments_rejected_on_host():
     assert L.fva_repair(None, 16, g, 1, 16, 16, 16, 16, None, 0, None) == fva.FVA_ERR_INVALID_ARG
     assert L.fva_repair(16, 16, g, 0, 16, 16, 16, 16, None, 0, None) == fva.FVA_ERR_INVALID_ARG
     assert L.fva_block_sparse_attn(16, 16, None, 16, 16, None, g, 0.0, 16, None) == fva.FVA_ERR_INVALID_ARG
+    assert L.fva_block_sparse_attn_natural(16, 16, 16, 16, 16, None, g, 0.0, None, None) == fva.FVA_ERR_INVALID_ARG
+    assert L.fva_block_sparse_attn_natural(16, 16, 16, 16, 16, None, _g(tt=1, ty=4, tx=8).c(), 0.0, 16, None) == \
+        fva.FVA_ERR_UNSUPPORTED
     t32 = _g(tt=1, ty=4, tx=8).c()                                            # 32-token tiles
     assert L.fva_block_sparse_attn(16, 16, 16, 16, 16, None, t32, 0.0, 16, None) == fva.FVA_ERR_UNSUPPORTED
     assert L.fva_block_sparse_attn(16, 16, 16, 16, 16, None, g, float("inf"), 16, None) == fva.FVA_ERR_INVALID_ARG
