@@ -223,6 +223,25 @@ def run_reference(args, rank: int, world: int):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ ranks ------------
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """The largest value of x over all ranks (every rank calls it; world 1: x itself).
+    Multi-rank times are taken this way: the job takes as long as its slowest rank."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world: int, units_per_rank: float, ms: float) -> float:
+    """Aggregate throughput of `world` replicas that each process units_per_rank in `ms`
+    (the max over ranks): weak scaling, units per second over the whole job."""
+    return world * units_per_rank / (ms * 1e-3)
+
+
 # ------------------------------------------------------------------ GPU arm ----------
 def run_gpu(args, rank: int, world: int, local_rank: int):
     import torch
@@ -290,11 +309,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
         torch.cuda.synchronize(dev)
     launches = fva.fva_launch_count() - launches0
     assert fva.fva_get_device_error(stream) == 0
-    total_ms = start.elapsed_time(stop)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(start.elapsed_time(stop), world, dev)
     ms = total_ms / K
     stage = np.array([[ev[s][i].elapsed_time(ev[s][i + 1]) for i in range(3)] for s in range(K)])
     st_mean = stage.mean(axis=0)            # reorder x3 (+ pooling), routing from the means, attention (ms)
@@ -329,11 +344,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
         outh.copy_(out, non_blocking=True)
     s1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = s0.elapsed_time(s1) / K
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(s0.elapsed_time(s1) / K, world, dev)
 
     if rank != 0:
         return
@@ -342,7 +353,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
     achieved = flops_actual / (attn_ms * 1e-3) / 1e12
     peak = peaks["bf16_tflops_sustained"]
     traffic = attn_traffic(cfg.name, pairs)
-    value = world * flops_actual / (ms * 1e-3) / 1e12
+    value = whole_job_rate(world, flops_actual, ms) / 1e12
     line = {
         "metric": METRIC,
         "value": value,
@@ -358,7 +369,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
         "data": "synthetic (seeded random-Fourier-feature Q/K, Gaussian V; stands in for Wan2.2 latents)",
         "config": dict(workload_desc(cfg), parallelism=f"replicas x{world} (no data-path collective)",
                        order="static" if args.static_order else "lpt"),
-        "dense_equiv_tflops": world * flops_dense / (ms * 1e-3) / 1e12,
+        "dense_equiv_tflops": whole_job_rate(world, flops_dense, ms) / 1e12,
         "attn_pct_bf16_peak": 100.0 * achieved / peak,
         "attn_pct_bf16_peak_burst": 100.0 * achieved / peaks["bf16_tflops"],
         "attn_kernel_tflops": achieved,
@@ -384,7 +395,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
                              "achieved": bytes_route / (fused_route_ms * 1e-3) / 1e9,
                              "peak": peaks["hbm_gbs"], "unit": "GB/s",
                              "frac": bytes_route / (fused_route_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]},
-        "e2e": {"value": world * flops_actual / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+        "e2e": {"value": whole_job_rate(world, flops_actual, e2e_ms) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": int(launches),
         "clocks": clk.summary(),
