@@ -13,7 +13,8 @@ CDF threshold with a Top-k safety floor, mask materialisation and runtime repair
 and then block-sparse attention.  Where the page is silent the readings are:
 
 * blocks are 3D box tiles of tt x ty x tx tokens, numbered in raster order of
-  the tile grid; tokens inside a tile are in raster order too;
+  the tile grid (or, with order="hilbert", along the Hilbert curve of the §3.1
+  overview, see tile_order); tokens inside a tile are in raster order;
 * "pooled" = arithmetic mean over the tile's tokens, in float64, of the
   bfloat16 inputs;
 * block importance = row softmax over key blocks of Qbar_i . Kbar_j / sqrt(d);
@@ -45,7 +46,7 @@ from typing import Iterable, Optional
 import numpy as np
 
 __all__ = [
-    "Geometry", "tile_source_index", "reorder", "inverse_reorder", "bf16_bits_to_f64",
+    "Geometry", "hilbert_index_3d", "tile_order", "tile_source_index", "reorder", "inverse_reorder", "bf16_bits_to_f64",
     "pool_blocks", "block_logits", "row_softmax", "rank_order", "topp_keep",
     "RouteResult", "route", "RepairResult", "repair", "lpt_worklist",
     "attention_items", "attention", "dense_attention", "tie_flags",
@@ -65,6 +66,7 @@ class Geometry:
     tt: int
     ty: int
     tx: int
+    order: str = "raster"   # numbering of the tiles: "raster" or "hilbert"
 
     @property
     def N(self) -> int:
@@ -83,24 +85,87 @@ class Geometry:
             raise ValueError("latent grid must be divisible by the tile")
 
     @staticmethod
-    def of(cfg) -> "Geometry":
-        return Geometry(cfg.B, cfg.H, cfg.T, cfg.Y, cfg.X, cfg.d, cfg.tt, cfg.ty, cfg.tx)
+    def of(cfg, order: str = "raster") -> "Geometry":
+        return Geometry(cfg.B, cfg.H, cfg.T, cfg.Y, cfg.X, cfg.d, cfg.tt, cfg.ty, cfg.tx, order)
 
 
 # --------------------------------------------------------------------------------------
 # Step 1: video-aware block organisation (abstract; §3.1 overview, block reordering).
 # --------------------------------------------------------------------------------------
+def hilbert_index_3d(c: tuple, bits: int) -> int:
+    """Position of grid cell c = (c0, c1, c2), each in [0, 2^bits), along the 3D Hilbert
+    curve of the 2^bits cube: Skilling's method ("Programming the Hilbert curve", 2004),
+    restated.  The coordinates are turned into the curve's "transposed" index: for each
+    bit level from the top, the lower bits are reflected or exchanged with the first
+    coordinate (undoing the curve's rotations), then the coordinates are Gray-coded;
+    the index is the transposed bits read level by level, c0 first."""
+    X = [int(v) for v in c]
+    n = 3
+    M = 1 << (bits - 1)
+    Q = M
+    while Q > 1:
+        P = Q - 1
+        for i in range(n):
+            if X[i] & Q:
+                X[0] ^= P
+            else:
+                t = (X[0] ^ X[i]) & P
+                X[0] ^= t
+                X[i] ^= t
+        Q >>= 1
+    for i in range(1, n):
+        X[i] ^= X[i - 1]
+    t = 0
+    Q = M
+    while Q > 1:
+        if X[n - 1] & Q:
+            t ^= Q - 1
+        Q >>= 1
+    for i in range(n):
+        X[i] ^= t
+    h = 0
+    for j in range(bits - 1, -1, -1):
+        for i in range(n):
+            h = (h << 1) | ((X[i] >> j) & 1)
+    return h
+
+
+def tile_order(g: Geometry) -> np.ndarray:
+    """order[b] = raster index of the tile numbered b.  Raster numbering is the identity.
+    Hilbert numbering (the §3.1 overview reorders blocks along a Hilbert curve so that
+    spatially adjacent tokens fall into nearby blocks): the tile grid (nT, nY, nX) sits
+    in the smallest 2^bits cube that holds it, and its tiles are numbered by ascending
+    Hilbert index of (bt, by, bx) in that cube (a generalisation to grids whose sides are
+    not powers of two: cells outside the grid are skipped)."""
+    g.check()
+    nT, nY, nX = g.T // g.tt, g.Y // g.ty, g.X // g.tx
+    if g.order == "raster":
+        return np.arange(nT * nY * nX, dtype=np.int64)
+    if g.order != "hilbert":
+        raise ValueError(f"unknown tile order {g.order!r}")
+    bits = max(1, int(max(nT, nY, nX) - 1).bit_length())
+    keys = []
+    for bt in range(nT):
+        for by in range(nY):
+            for bx in range(nX):
+                keys.append((hilbert_index_3d((bt, by, bx), bits), (bt * nY + by) * nX + bx))
+    keys.sort()
+    return np.array([r for _, r in keys], dtype=np.int64)
+
+
 def tile_source_index(g: Geometry) -> np.ndarray:
     """src[n'] = natural token index n of the token placed at reordered position n'.
 
-    Position n' = b * S + r, with b the raster index of the tile over the tile
-    grid (T/tt, Y/ty, X/tx) and r the raster index of the token inside the tile
-    over (tt, ty, tx).  The natural index is n = (t * Y + y) * X + x.
+    Position n' = b * S + r, with b the number of the tile (tile_order: raster index of
+    the tile over the tile grid (T/tt, Y/ty, X/tx), or its Hilbert rank) and r the raster
+    index of the token inside the tile over (tt, ty, tx).  The natural index is
+    n = (t * Y + y) * X + x.
     """
     g.check()
     nT, nY, nX = g.T // g.tt, g.Y // g.ty, g.X // g.tx
     npos = np.arange(g.N, dtype=np.int64)
     b, r = np.divmod(npos, g.S)
+    b = tile_order(g)[b]
     bt, rem = np.divmod(b, nY * nX)
     by, bx = np.divmod(rem, nX)
     lt, rem = np.divmod(r, g.ty * g.tx)

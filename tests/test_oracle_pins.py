@@ -2,6 +2,7 @@
 than itself (hand-derived fixtures, brute force, library routines, closed forms,
 invariants), so that a dropped term, a wrong sign, index or transposed operand
 fails at least one of them.  CPU only."""
+import dataclasses
 import itertools
 import json
 import math
@@ -350,3 +351,53 @@ def test_generator_head_scales():
     assert (a[0::2] == 4.0).all() and (a[1::2] == 0.3).all()
     lu = synth.head_scales(synth.CONFIGS["wan480p"], np.linspace(0, 1, 40))
     assert math.isclose(lu[0], 0.5) and math.isclose(lu[-1], 4.0)
+
+
+# ----------------------------------------------------------------- Hilbert tile numbering
+def test_hilbert_2x2x2_matches_hand_derivation():
+    fx = json.load(open(os.path.join(GOLDEN, "hilbert_fixture.json")))
+    for h, c in enumerate(fx["cells_in_order"]):
+        assert O.hilbert_index_3d(tuple(c), fx["bits"]) == h
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3])
+def test_hilbert_cube_is_a_face_adjacent_path(bits):
+    side = 1 << bits
+    idx = {}
+    for c in itertools.product(range(side), repeat=3):
+        idx[O.hilbert_index_3d(c, bits)] = c
+    assert sorted(idx) == list(range(side ** 3))          # a bijection onto [0, side^3)
+    assert idx[0] == (0, 0, 0)
+    for h in range(1, side ** 3):                        # consecutive cells share a face
+        a, b = idx[h - 1], idx[h]
+        assert sum(abs(x - y) for x, y in zip(a, b)) == 1, (h, a, b)
+
+
+def test_tile_order_raster_is_identity_and_hilbert_a_permutation():
+    g = O.Geometry(1, 1, 20, 32, 48, 64, 2, 8, 8)
+    assert np.array_equal(O.tile_order(g), np.arange(240))
+    gh = dataclasses.replace(g, order="hilbert")
+    o = O.tile_order(gh)
+    assert sorted(o.tolist()) == list(range(240)) and not np.array_equal(o, np.arange(240))
+    # a power-of-two grid: consecutive tiles are face neighbours
+    g8 = O.Geometry(1, 1, 8, 32, 32, 64, 2, 8, 8, "hilbert")      # 4 x 4 x 4 tiles
+    o8 = O.tile_order(g8)
+    for a, b in zip(o8[:-1], o8[1:]):
+        ca, cb = np.unravel_index(a, (4, 4, 4)), np.unravel_index(b, (4, 4, 4))
+        assert sum(abs(int(x) - int(y)) for x, y in zip(ca, cb)) == 1
+
+
+def test_reorder_with_hilbert_numbering():
+    g = O.Geometry(1, 2, 4, 16, 24, 64, 2, 8, 8, "hilbert")       # 2 x 2 x 3 tiles
+    x = np.random.default_rng(5).integers(0, 1 << 16, size=(1, 2, g.N, 64), dtype=np.uint16)
+    xr = O.reorder(x, g)
+    assert np.array_equal(O.inverse_reorder(xr, g), x)
+    src = O.tile_source_index(g)
+    order = O.tile_order(g)
+    nY, nX = g.Y // g.ty, g.X // g.tx
+    for b in range(g.Nb):   # block b holds exactly the tokens of tile order[b], in raster order
+        bt, rem = divmod(int(order[b]), nY * nX)
+        by, bx = divmod(rem, nX)
+        want = [((bt * g.tt + lt) * g.Y + by * g.ty + ly) * g.X + bx * g.tx + lx
+                for lt in range(g.tt) for ly in range(g.ty) for lx in range(g.tx)]
+        assert src[b * g.S:(b + 1) * g.S].tolist() == want
