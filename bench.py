@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(synth.CONFIGS))
     ap.add_argument("--impl", default="fva", choices=["fva", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tile-order", choices=("raster", "hilbert"), default="raster",
+                    help="tile numbering: raster, or along the 3D Hilbert curve")
     ap.add_argument("--static-order", action="store_true", help="item-id order instead of the LPT work list")
     ap.add_argument("--report", choices=["stress", "sweep"], default=None,
                     help="instead of the headline line: head-heterogeneity stress (LPT vs item-id order) or the "
@@ -252,6 +254,8 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
     dev = torch.device("cuda", local_rank)
     cfg = synth.CONFIGS[args.config]
     g = fva.Geom.of(cfg)
+    if args.tile_order == "hilbert":
+        g = g.with_tiles(fva.FVA_TILES_HILBERT, device=dev)
     peaks = load_peaks()
 
     q, k, v = synth.make_qkv(cfg)
@@ -368,7 +372,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
         "dtype": "bf16",
         "data": "synthetic (seeded random-Fourier-feature Q/K, Gaussian V; stands in for Wan2.2 latents)",
         "config": dict(workload_desc(cfg), parallelism=f"replicas x{world} (no data-path collective)",
-                       order="static" if args.static_order else "lpt"),
+                       order="static" if args.static_order else "lpt", tiles=args.tile_order),
         "dense_equiv_tflops": whole_job_rate(world, flops_dense, ms) / 1e12,
         "attn_pct_bf16_peak": 100.0 * achieved / peak,
         "attn_pct_bf16_peak_burst": 100.0 * achieved / peaks["bf16_tflops"],

@@ -34,7 +34,11 @@ class FvaError(RuntimeError):
 
 
 class _Geom(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_int32) for n in ("B", "H", "T", "Y", "X", "d", "tt", "ty", "tx")]
+    _fields_ = [(n, ctypes.c_int32) for n in ("B", "H", "T", "Y", "X", "d", "tt", "ty", "tx")] + \
+               [("tile_order", ctypes.c_void_p)]
+
+
+FVA_TILES_RASTER, FVA_TILES_HILBERT = 0, 1
 
 
 @dataclasses.dataclass(frozen=True)
@@ -50,6 +54,7 @@ class Geom:
     tt: int
     ty: int
     tx: int
+    tile_order: Optional[torch.Tensor] = dataclasses.field(default=None, compare=False)  # device int32 [Nb]
 
     @property
     def N(self) -> int:
@@ -64,11 +69,17 @@ class Geom:
         return self.N // self.S
 
     def c(self) -> _Geom:
-        return _Geom(self.B, self.H, self.T, self.Y, self.X, self.d, self.tt, self.ty, self.tx)
+        order = None if self.tile_order is None else self.tile_order.data_ptr()
+        return _Geom(self.B, self.H, self.T, self.Y, self.X, self.d, self.tt, self.ty, self.tx, order)
 
     @staticmethod
     def of(cfg) -> "Geom":
         return Geom(cfg.B, cfg.H, cfg.T, cfg.Y, cfg.X, cfg.d, cfg.tt, cfg.ty, cfg.tx)
+
+    def with_tiles(self, kind: int, device="cuda") -> "Geom":
+        """This geometry with the tile numbering `kind` (FVA_TILES_RASTER / _HILBERT) as a device table."""
+        table = fva_tile_order(self, kind)
+        return dataclasses.replace(self, tile_order=torch.from_numpy(table).to(device))
 
 
 def _load():
@@ -79,6 +90,7 @@ def _load():
                                   ctypes.c_float, ctypes.c_double)
     sig = {
         "fva_reorder": ([vp, vp, _Geom, vp], ctypes.c_int),
+        "fva_tile_order": ([_Geom, i32, vp], ctypes.c_int),
         "fva_inverse_reorder": ([vp, vp, _Geom, vp], ctypes.c_int),
         "fva_route_workspace_size": ([_Geom], sz),
         "fva_route": ([vp, vp, _Geom, f64, i32, vp, vp, vp, vp, sz, vp], ctypes.c_int),
@@ -136,6 +148,15 @@ def _need(t: torch.Tensor, dtype: torch.dtype, shape, name: str) -> None:
 
 
 # ------------------------------------------------------------------ 1:1 wrappers ----
+def fva_tile_order(g: Geom, kind: int):
+    """Host table of a tile numbering: order[b] = raster index of the tile numbered b."""
+    import numpy as np
+    out = np.empty(g.Nb, dtype=np.int32)
+    _check(lib.fva_tile_order(dataclasses.replace(g, tile_order=None).c(), int(kind),
+                              out.ctypes.data_as(ctypes.c_void_p)))
+    return out
+
+
 def fva_reorder(x: torch.Tensor, xr: torch.Tensor, g: Geom, stream=None) -> None:
     shp = (g.B, g.H, g.N, g.d)
     _need(x, torch.bfloat16, shp, "x")

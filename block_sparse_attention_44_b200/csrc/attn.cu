@@ -90,14 +90,17 @@ struct AttnParams {
   // natural != 0: row r of tile i is written at its natural token position (the inverse
   // reorder fused into the epilogue); grid X, Y and tile tt x ty x tx, nY x nX tiles
   int natural, Y, X, tt, ty, tx, nY, nX;
+  const int32_t* order;   // tile numbering table (raster index of tile i), or nullptr
 };
 
 // Token position of row r of tile i in the output: tile-major i*S + r, or the natural
-// raster index of that token when prm.natural is set.
+// raster index of that token when prm.natural is set (-1: bad numbering table entry).
 __device__ __forceinline__ long long out_token(const AttnParams& prm, int i, int r, int S) {
   if (!prm.natural) return static_cast<long long>(i) * S + r;
-  const int bt = i / (prm.nY * prm.nX);
-  const int rem = i - bt * prm.nY * prm.nX;
+  const int tr = prm.order ? prm.order[i] : i;
+  if (tr < 0 || tr >= prm.Nb) return -1;
+  const int bt = tr / (prm.nY * prm.nX);
+  const int rem = tr - bt * prm.nY * prm.nX;
   const int by = rem / prm.nX;
   const int bx = rem - by * prm.nX;
   const int tyx = prm.ty * prm.tx;
@@ -408,9 +411,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int n = item_count(prm, item);
       const long long bh = item / Nb;
       const int i = item - static_cast<int>(bh * Nb);
-      uint16_t* orow = prm.out + (bh * prm.N + out_token(prm, i, row < S ? row : 0, S)) * D + half * HD;
+      const long long tok = out_token(prm, i, row < S ? row : 0, S);
+      if (tok < 0) set_device_error(prm.dev_err, kDevErrBadIndex);
+      uint16_t* orow = prm.out + (bh * prm.N + (tok < 0 ? 0 : tok)) * D + half * HD;
+      const bool wr = row < S && tok >= 0;   // this thread writes its row
       if (n <= 0) {
-        if (row < S)
+        if (wr)
           for (int c = 0; c < HD; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
         continue;
       }
@@ -517,7 +523,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
         for (int e = 0; e < 16; ++e)
           pk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
-        if (row < S) {
+        if (wr) {
           uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
           for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
@@ -626,6 +632,7 @@ cudaError_t launch_attention(const void* qr, const void* kr, const void* vr, con
   prm.tx = natural ? natural->tx : 0;
   prm.nY = D.nY;
   prm.nX = D.nX;
+  prm.order = natural ? D.order : nullptr;
   cudaError_t e;
   if (D.d == 128 && D.S == 128)
     e = launch_t<128, 128, 3, 3>(mq, mk, mv, prm, s);

@@ -4,7 +4,10 @@
 #include <stdarg.h>
 #include <stdio.h>
 
+#include <algorithm>
 #include <atomic>
+#include <utility>
+#include <vector>
 
 #include "fva_common.cuh"
 #include "fva_internal.h"
@@ -66,7 +69,42 @@ int check_geom(const fva_geom& g, fva::Dims& D, bool need_attn_shapes) {
   D.nT = g.T / g.tt;
   D.nY = g.Y / g.ty;
   D.nX = g.X / g.tx;
+  D.order = g.tile_order;
+  if ((reinterpret_cast<uintptr_t>(g.tile_order) & 3u) != 0)
+    return fail(FVA_ERR_INVALID_ARG, "tile_order must be 4-byte aligned");
   return FVA_OK;
+}
+
+// Position of cell c (each coordinate < 2^bits) along the 3D Hilbert curve of the
+// 2^bits cube, by Skilling's transposed-index construction: from the top bit level
+// down, undo the curve's rotations (reflect or exchange the lower bits with the first
+// coordinate), Gray-code the coordinates, then read the transposed bits level by
+// level, first coordinate first.
+unsigned long long hilbert_index_3d(const unsigned (&c)[3], int bits) {
+  unsigned x[3] = {c[0], c[1], c[2]};
+  const unsigned top = 1u << (bits - 1);
+  for (unsigned q = top; q > 1; q >>= 1) {
+    const unsigned low = q - 1;
+    for (int i = 0; i < 3; ++i) {
+      if (x[i] & q) {
+        x[0] ^= low;
+      } else {
+        const unsigned t = (x[0] ^ x[i]) & low;
+        x[0] ^= t;
+        x[i] ^= t;
+      }
+    }
+  }
+  x[1] ^= x[0];
+  x[2] ^= x[1];
+  unsigned flip = 0;
+  for (unsigned q = top; q > 1; q >>= 1)
+    if (x[2] & q) flip ^= q - 1;
+  for (unsigned& v : x) v ^= flip;
+  unsigned long long h = 0;
+  for (int j = bits - 1; j >= 0; --j)
+    for (int i = 0; i < 3; ++i) h = (h << 1) | ((x[i] >> j) & 1u);
+  return h;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -82,11 +120,44 @@ int finish(cudaError_t e, int launches, const char* where) {
 
 extern "C" {
 
-int32_t fva_version(void) { return 103; }
+int32_t fva_version(void) { return 104; }
 
 const char* fva_last_error(void) { return g_err; }
 
 int64_t fva_launch_count(void) { return g_launches.load(); }
+
+int fva_tile_order(fva_geom g, int32_t kind, int32_t* order_out) {
+  fva::Dims D;
+  int rc = check_geom(g, D, false);
+  if (rc) return rc;
+  if (!order_out) return fail(FVA_ERR_INVALID_ARG, "null pointer");
+  const int n = D.Nb;
+  if (kind == FVA_TILES_RASTER) {
+    for (int b = 0; b < n; ++b) order_out[b] = b;
+    g_err[0] = '\0';
+    return FVA_OK;
+  }
+  if (kind != FVA_TILES_HILBERT) return fail(FVA_ERR_INVALID_ARG, "unknown tile numbering %d", kind);
+  int side = 1, bits = 0;
+  const int m = D.nT > D.nY ? (D.nT > D.nX ? D.nT : D.nX) : (D.nY > D.nX ? D.nY : D.nX);
+  while (side < m) {
+    side <<= 1;
+    ++bits;
+  }
+  if (bits == 0) bits = 1;
+  std::vector<std::pair<unsigned long long, int>> keys;
+  keys.reserve(n);
+  for (int bt = 0; bt < D.nT; ++bt)
+    for (int by = 0; by < D.nY; ++by)
+      for (int bx = 0; bx < D.nX; ++bx) {
+        const unsigned c[3] = {static_cast<unsigned>(bt), static_cast<unsigned>(by), static_cast<unsigned>(bx)};
+        keys.emplace_back(hilbert_index_3d(c, bits), (bt * D.nY + by) * D.nX + bx);
+      }
+  std::sort(keys.begin(), keys.end());
+  for (int b = 0; b < n; ++b) order_out[b] = keys[b].second;
+  g_err[0] = '\0';
+  return FVA_OK;
+}
 
 static int reorder_common(const void* src, void* dst, fva_geom g, void* stream, bool inverse) {
   fva::Dims D;
@@ -95,8 +166,10 @@ static int reorder_common(const void* src, void* dst, fva_geom g, void* stream, 
   if (!src || !dst) return fail(FVA_ERR_INVALID_ARG, "null tensor pointer");
   if (src == dst) return fail(FVA_ERR_INVALID_ARG, "in-place reorder is not supported");
   if (!aligned16(src) || !aligned16(dst)) return fail(FVA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  int* de = dev_err_ptr();
+  if (!de) return fail(FVA_ERR_CUDA, "reorder: cannot resolve the device error word");
   int launches = 0;
-  cudaError_t e = fva::launch_reorder(src, dst, g, D, inverse, static_cast<cudaStream_t>(stream), &launches);
+  cudaError_t e = fva::launch_reorder(src, dst, g, D, inverse, de, static_cast<cudaStream_t>(stream), &launches);
   return finish(e, launches, inverse ? "fva_inverse_reorder" : "fva_reorder");
 }
 
@@ -114,8 +187,10 @@ int fva_reorder_pool(const void* x, void* xr, double* pooled, fva_geom g, void* 
   if (x == xr) return fail(FVA_ERR_INVALID_ARG, "in-place reorder is not supported");
   if (!aligned16(x) || !aligned16(xr)) return fail(FVA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
   if ((reinterpret_cast<uintptr_t>(pooled) & 7u) != 0) return fail(FVA_ERR_INVALID_ARG, "pooled must be 8-byte aligned");
+  int* de = dev_err_ptr();
+  if (!de) return fail(FVA_ERR_CUDA, "fva_reorder_pool: cannot resolve the device error word");
   int launches = 0;
-  cudaError_t e = fva::launch_reorder_pool(x, xr, pooled, g, D, static_cast<cudaStream_t>(stream), &launches);
+  cudaError_t e = fva::launch_reorder_pool(x, xr, pooled, g, D, de, static_cast<cudaStream_t>(stream), &launches);
   return finish(e, launches, "fva_reorder_pool");
 }
 

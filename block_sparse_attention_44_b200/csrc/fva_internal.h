@@ -11,6 +11,7 @@ namespace fva {
 // Derived sizes of a validated geometry.
 struct Dims {
   int B, H, N, d, S, Nb, nT, nY, nX;
+  const int32_t* order;   // tile numbering (device, Nb entries) or nullptr for raster
   long long BH() const { return static_cast<long long>(B) * H; }
   long long rows() const { return BH() * Nb; }   // (b, h, query-block) rows / work items
 };
@@ -19,11 +20,11 @@ constexpr int kMaxNb = 2048;
 
 // Reorder / inverse reorder of one bf16 [B,H,N,d] tensor.
 cudaError_t launch_reorder(const void* src, void* dst, const fva_geom& g, const Dims& D, bool inverse,
-                           cudaStream_t s, int* launches);
+                           int* dev_err, cudaStream_t s, int* launches);
 
 // Forward reorder that also writes the float64 mean of every tile ([B*H*Nb, d]).
 cudaError_t launch_reorder_pool(const void* src, void* dst, double* pooled, const fva_geom& g, const Dims& D,
-                                cudaStream_t s, int* launches);
+                                int* dev_err, cudaStream_t s, int* launches);
 
 // Routing: block means (float64), float64 logits, Top-p / Top-k selection; with
 // counts != nullptr also the repaired, compacted per-row lists (idx, counts).

@@ -2,12 +2,14 @@
 // order ("FVAttn: Adaptive Sparse Attention with Runtime Load Balancing for Video
 // Generation", abstract and §3.1 overview; tiles are raster-numbered boxes).
 //
-// One CTA moves one tile of one (b, h): S rows of d bf16.  On the natural side a
-// tile is tt*ty runs of tx consecutive tokens (tx*d*2 contiguous bytes each), on
-// the tile-major side it is one contiguous S*d*2-byte block, so both sides stream
-// whole 32-byte sectors with 16-byte vector accesses.  Pure HBM copy: 2*S*d*2
-// bytes of traffic per CTA.  reorder_pool_kernel also writes the tile's float64 mean
-// (the routing pool step riding on the same pass: no second read of Q or K).
+// One CTA moves one tile of one (b, h): S rows of d bf16.  The tile numbered b is
+// raster tile b, or tile order[b] when a numbering table is given (Hilbert
+// numbering).  On the natural side a tile is tt*ty runs of tx consecutive tokens
+// (tx*d*2 contiguous bytes each), on the tile-major side it is one contiguous
+// S*d*2-byte block, so both sides stream whole 32-byte sectors with 16-byte vector
+// accesses.  Pure HBM copy: 2*S*d*2 bytes of traffic per CTA.  reorder_pool_kernel
+// also writes the tile's float64 mean (the routing pool step riding on the same pass:
+// no second read of Q or K).
 #include "fva_common.cuh"
 #include "fva_internal.h"
 
@@ -20,15 +22,21 @@ template <int D>
 __global__ void __launch_bounds__(kReorderThreads) reorder_kernel(const uint4* __restrict__ src,
                                                                   uint4* __restrict__ dst, int N, int Y, int X,
                                                                   int tt, int ty, int tx, int nY, int nX, int S,
-                                                                  int Nb, int inverse) {
+                                                                  int Nb, int inverse, const int32_t* __restrict__ order,
+                                                                  int* dev_err) {
   constexpr int CPR = D * 2 / 16;   // 16-byte chunks per token row
   constexpr int U = 8;              // chunks in flight per thread
   extern __shared__ int nat_row[];  // natural token index of tile row r
   const long long blk = blockIdx.x;
   const long long bh = blk / Nb;
   const int b = static_cast<int>(blk - bh * Nb);
-  const int bt = b / (nY * nX);
-  const int rem = b - bt * nY * nX;
+  const int tr = order ? order[b] : b;   // raster index of the tile numbered b
+  if (tr < 0 || tr >= Nb) {
+    if (threadIdx.x == 0) set_device_error(dev_err, kDevErrBadIndex);
+    return;
+  }
+  const int bt = tr / (nY * nX);
+  const int rem = tr - bt * nY * nX;
   const int by = rem / nX;
   const int bx = rem - by * nX;
   const int tyx = ty * tx;
@@ -77,7 +85,8 @@ __global__ void __launch_bounds__(kReorderThreads) reorder_pool_kernel(const uin
                                                                        uint4* __restrict__ dst,
                                                                        double* __restrict__ pooled, int N, int Y,
                                                                        int X, int tt, int ty, int tx, int nY, int nX,
-                                                                       int S, int Nb) {
+                                                                       int S, int Nb, const int32_t* __restrict__ order,
+                                                                       int* dev_err) {
   constexpr int CPR = D * 2 / 16;            // 16-byte chunks per token row
   constexpr int RG = kReorderThreads / CPR;  // row groups
   constexpr int U = 8;                       // rows in flight per thread
@@ -86,8 +95,13 @@ __global__ void __launch_bounds__(kReorderThreads) reorder_pool_kernel(const uin
   const long long blk = blockIdx.x;
   const long long bh = blk / Nb;
   const int b = static_cast<int>(blk - bh * Nb);
-  const int bt = b / (nY * nX);
-  const int rem = b - bt * nY * nX;
+  const int tr = order ? order[b] : b;   // raster index of the tile numbered b
+  if (tr < 0 || tr >= Nb) {
+    if (threadIdx.x == 0) set_device_error(dev_err, kDevErrBadIndex);
+    return;
+  }
+  const int bt = tr / (nY * nX);
+  const int rem = tr - bt * nY * nX;
   const int by = rem / nX;
   const int bx = rem - by * nX;
   const int tyx = ty * tx;
@@ -139,33 +153,35 @@ __global__ void __launch_bounds__(kReorderThreads) reorder_pool_kernel(const uin
 }  // namespace
 
 cudaError_t launch_reorder_pool(const void* src, void* dst, double* pooled, const fva_geom& g, const Dims& D,
-                                cudaStream_t s, int* launches) {
+                                int* dev_err, cudaStream_t s, int* launches) {
   const dim3 grid(static_cast<unsigned>(D.rows()));
   const size_t smem = static_cast<size_t>(D.S) * sizeof(int);
   if (D.d == 128)
     reorder_pool_kernel<128><<<grid, kReorderThreads, smem, s>>>(static_cast<const uint4*>(src),
                                                                  static_cast<uint4*>(dst), pooled, D.N, g.Y, g.X,
-                                                                 g.tt, g.ty, g.tx, D.nY, D.nX, D.S, D.Nb);
+                                                                 g.tt, g.ty, g.tx, D.nY, D.nX, D.S, D.Nb, D.order,
+                                                                 dev_err);
   else
     reorder_pool_kernel<64><<<grid, kReorderThreads, smem, s>>>(static_cast<const uint4*>(src),
                                                                 static_cast<uint4*>(dst), pooled, D.N, g.Y, g.X,
-                                                                g.tt, g.ty, g.tx, D.nY, D.nX, D.S, D.Nb);
+                                                                g.tt, g.ty, g.tx, D.nY, D.nX, D.S, D.Nb, D.order,
+                                                                dev_err);
   ++*launches;
   return cudaGetLastError();
 }
 
 cudaError_t launch_reorder(const void* src, void* dst, const fva_geom& g, const Dims& D, bool inverse,
-                           cudaStream_t s, int* launches) {
+                           int* dev_err, cudaStream_t s, int* launches) {
   const dim3 grid(static_cast<unsigned>(D.rows()));
   const size_t smem = static_cast<size_t>(D.S) * sizeof(int);
   if (D.d == 128) {
     reorder_kernel<128><<<grid, kReorderThreads, smem, s>>>(
         static_cast<const uint4*>(src), static_cast<uint4*>(dst), D.N, g.Y, g.X, g.tt, g.ty, g.tx, D.nY, D.nX, D.S,
-        D.Nb, inverse ? 1 : 0);
+        D.Nb, inverse ? 1 : 0, D.order, dev_err);
   } else {
     reorder_kernel<64><<<grid, kReorderThreads, smem, s>>>(
         static_cast<const uint4*>(src), static_cast<uint4*>(dst), D.N, g.Y, g.X, g.tt, g.ty, g.tx, D.nY, D.nX, D.S,
-        D.Nb, inverse ? 1 : 0);
+        D.Nb, inverse ? 1 : 0, D.order, dev_err);
   }
   ++*launches;
   return cudaGetLastError();

@@ -50,10 +50,32 @@ enum {
   FVA_ERR_TIMEOUT = 4        /* a bounded device-side wait expired (reported by fva_get_device_error) */
 };
 
-/* Problem geometry: batch B, heads H, latent grid T x Y x X, head_dim d, tile tt x ty x tx. */
+/*
+ * Problem geometry: batch B, heads H, latent grid T x Y x X, head_dim d, tile tt x ty x tx.
+ * tile_order: NULL for raster numbering of the tiles, else a DEVICE int32 array of Nb
+ * entries, tile_order[b] = raster index (bt * nY + by) * nX + bx of the tile numbered b
+ * (a permutation of [0, Nb), e.g. the Hilbert numbering from fva_tile_order).  Only the
+ * token permutation uses it: fva_reorder, fva_reorder_pool, fva_inverse_reorder and
+ * fva_block_sparse_attn_natural; an entry outside [0, Nb) raises device error 2 and its
+ * tile is skipped.
+ */
 typedef struct fva_geom {
   int32_t B, H, T, Y, X, d, tt, ty, tx;
+  const int32_t* tile_order;
 } fva_geom;
+
+enum { FVA_TILES_RASTER = 0, FVA_TILES_HILBERT = 1 };
+
+/*
+ * fva_tile_order — host-side table of a tile numbering (§3.1 overview: blocks are
+ * reordered along a Hilbert curve so that spatially adjacent tokens fall into nearby
+ * blocks).  order_out (HOST, Nb int32) receives the raster index of the tile numbered
+ * b.  FVA_TILES_HILBERT: the tile grid (nT, nY, nX) is placed in the smallest
+ * power-of-two cube holding it and its tiles are numbered by ascending 3D Hilbert index
+ * of (bt, by, bx) in that cube (Skilling's transposed-index construction); the caller
+ * copies the table to the device and passes it as g.tile_order.  No GPU work.
+ */
+int fva_tile_order(fva_geom g, int32_t kind, int32_t* order_out);
 
 /*
  * fva_reorder — video-aware block organisation (abstract; §3.1 overview, block

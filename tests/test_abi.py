@@ -120,3 +120,20 @@ def test_python_wrapper_type_checks():
     x = torch.zeros((1, 2, 256, 64), dtype=torch.float32)
     with pytest.raises(TypeError):
         fva.fva_reorder(x, x, g)
+
+
+def test_tile_order_table_matches_oracle():
+    import numpy as np
+
+    import oracle as O
+    for (T, Y, X, tt, ty, tx) in [(20, 32, 48, 2, 8, 8), (20, 48, 80, 2, 8, 8), (3, 5, 7, 1, 1, 1),
+                                  (8, 32, 32, 2, 8, 8), (1, 8, 8, 1, 8, 8), (6, 40, 24, 2, 8, 8)]:
+        g = fva.Geom(1, 1, T, Y, X, 64, tt, ty, tx)
+        want = O.tile_order(O.Geometry(1, 1, T, Y, X, 64, tt, ty, tx, "hilbert"))
+        assert np.array_equal(fva.fva_tile_order(g, fva.FVA_TILES_HILBERT), want)
+        assert np.array_equal(fva.fva_tile_order(g, fva.FVA_TILES_RASTER), np.arange(g.Nb))
+    with pytest.raises(fva.FvaError):
+        fva.fva_tile_order(_g(), 7)
+    bad = _g().c()
+    bad.tile_order = 18                                   # not 4-byte aligned
+    assert fva.lib.fva_reorder(16, 32, bad, None) == fva.FVA_ERR_INVALID_ARG

@@ -44,7 +44,10 @@ CASES = {
     "topk_only": _cfg("topk_only", H=3, T=4, Y=16, X=32, p=1e-9, k=3, seed=6),
     "k_above_nb": _cfg("k_above_nb", H=2, T=4, Y=16, X=16, k=50, seed=7),
     "single_block": _cfg("single_block", H=2, T=2, Y=8, X=8, seed=8),
+    # Hilbert numbering of a 3 x 3 x 5 tile grid (non-power-of-two sides)
+    "d128_hilbert": _cfg("d128_hilbert", B=1, H=4, T=6, Y=24, X=40, seed=9),
 }
+HILBERT = {"d128_hilbert"}
 
 
 @pytest.mark.parametrize("name", list(CASES))
@@ -52,6 +55,9 @@ def test_path_matches_oracle(fva, name):
     cfg = CASES[name]
     g = fva.Geom.of(cfg)
     og = O.Geometry.of(cfg)
+    if name in HILBERT:
+        g = g.with_tiles(fva.FVA_TILES_HILBERT)
+        og = O.Geometry.of(cfg, "hilbert")
     q, k, v = synth.make_qkv(cfg)
     dev = run_path(fva, g, q, k, v, cfg.p, cfg.k, want_logits=True)
 
@@ -125,6 +131,61 @@ def test_route_wide_rows(fva, name):
     # 1e-5 band around p flags about 2e-5 * Nb of such rows (2.4 % at Nb = 700)
     check_route(rr, mask_dev, topk_dev, max_tie_frac=0.05)
     check_repair(dict(counts=counts, idx=idx, head_work=hw, worklist=wl), mask_dev, topk_dev)
+
+
+def test_hilbert_numbering_keeps_the_token_pairs(fva):
+    """Renumbering the tiles renames blocks only: the kept (query tile, key tile) pairs,
+    mapped back to raster tile ids, are those of the raster numbering except on rows
+    either routing flags as ties (block-id tie-breaks depend on the numbering)."""
+    cfg = CASES["d128_hilbert"]
+    q, k, v = synth.make_qkv(cfg)
+    kept, flagged = {}, {}
+    for kind, order in ((fva.FVA_TILES_RASTER, "raster"), (fva.FVA_TILES_HILBERT, "hilbert")):
+        g = fva.Geom.of(cfg).with_tiles(kind)
+        og = O.Geometry.of(cfg, order)
+        dev = run_path(fva, g, q, k, v, cfg.p, cfg.k)
+        rr = O.route(O.reorder(q, og), O.reorder(k, og), og, cfg.p, cfg.k)
+        t1, t2p, t2k = O.tie_flags(rr)
+        tab = O.tile_order(og)
+        counts = dev["counts"].cpu().numpy()
+        idx = dev["idx"].cpu().numpy()
+        pairs = set()
+        rows = set()
+        for h in range(cfg.H):
+            for i in range(og.Nb):
+                for j in idx[0, h, i, :counts[0, h, i]]:
+                    pairs.add((h, int(tab[i]), int(tab[j])))
+                if t1[0, h, i] or t2p[0, h, i] or t2k[0, h, i]:
+                    rows.add((h, int(tab[i])))
+        kept[order], flagged[order] = pairs, rows
+    ties = flagged["raster"] | flagged["hilbert"]
+    strip = lambda s: {p for p in s if (p[0], p[1]) not in ties}
+    assert strip(kept["raster"]) == strip(kept["hilbert"])
+    assert len(ties) <= 0.05 * cfg.H * 45
+
+
+def test_bad_tile_numbering_entry_is_reported(fva):
+    cfg = CASES["d128_hilbert"]
+    g = fva.Geom.of(cfg).with_tiles(fva.FVA_TILES_HILBERT)
+    bad = g.tile_order.clone()
+    bad[3] = g.Nb + 7                                  # outside [0, Nb): the tile is skipped
+    gb = fva.Geom.of(cfg)
+    import dataclasses
+    gb = dataclasses.replace(gb, tile_order=bad)
+    q, _, _ = synth.make_qkv(cfg)
+    qd = to_dev(q)
+    out = torch.zeros_like(qd)
+    fva.fva_reorder(qd, out, gb)
+    assert fva.fva_get_device_error() == 2
+    good = torch.zeros_like(qd)
+    fva.fva_reorder(qd, good, g)
+    torch.cuda.synchronize()
+    S = g.S                                           # every other tile was written as usual
+    keep = torch.ones(g.Nb, dtype=torch.bool)
+    keep[3] = False
+    rows = keep.repeat_interleave(S).cuda()
+    assert torch.equal(out[:, :, rows].view(torch.int16), good[:, :, rows].view(torch.int16))
+    assert fva.fva_get_device_error() == 0
 
 
 def test_lpt_and_static_order_identical(fva):
