@@ -41,6 +41,7 @@ closed forms and invariants.
 from __future__ import annotations
 
 import dataclasses
+import math
 from typing import Iterable, Optional
 
 import numpy as np
@@ -49,7 +50,7 @@ __all__ = [
     "Geometry", "hilbert_index_3d", "tile_order", "tile_source_index", "reorder", "inverse_reorder", "bf16_bits_to_f64",
     "pool_blocks", "block_logits", "row_softmax", "rank_order", "topp_keep",
     "RouteResult", "route", "RepairResult", "repair", "lpt_worklist",
-    "attention_items", "attention", "dense_attention", "tie_flags",
+    "attention_items", "attention", "dense_attention", "tie_flags", "sasa_extend", "sasa_augment",
 ]
 
 
@@ -326,6 +327,68 @@ def repair(topp_mask: np.ndarray, topk_idx: np.ndarray) -> RepairResult:
 # Step 4: block-sparse attention over the kept blocks (§3.1 overview, last
 # compute stage; §2 background: only the selected block pairs are evaluated).
 # --------------------------------------------------------------------------------------
+# --------------------------------------------------------------------------------------
+# Slack-aware augmentation, single-GPU reading (§3.3 SASA; the formulas are garbled in the
+# page text, the readings are stated here).  The heads are split into num_ranks virtual
+# ranks of H / num_ranks consecutive heads (the Ulysses head layout of §2); W_r = sum of
+# W_h over the rank's heads and batch items; W* = max_r W_r is the critical path; rank r
+# gets the extra budget B_r = floor(alpha * (W* - W_r)) block pairs (alpha: the
+# augmentation coefficient, 0 <= alpha <= 1, so W_r + B_r <= W*).  B_r is spread over
+# the rank's rows, in item order u = (b*H + h)*Nb + i, round-robin: q = B_r // n_rows
+# extra positions each, one more for the first B_r % n_rows rows.  A row extends its
+# ranked prefix (the Top-p set with the floor, max(n_p, min(k, Nb)) blocks, following the
+# routing's importance order) by its share, capped at Nb: the kept set becomes the first
+# min(Nb, prefix + share) ranked blocks plus the diagonal.
+# --------------------------------------------------------------------------------------
+def sasa_extend(prefix: np.ndarray, head_work: np.ndarray, num_ranks: int, alpha: float) -> np.ndarray:
+    """New ranked-prefix length of every row: prefix int [B, H, Nb] (max(n_p, kk) per row),
+    head_work int [B, H] (W_h of the current lists).  Returns int64 [B, H, Nb]."""
+    B, H, Nb = prefix.shape
+    if num_ranks < 1 or H % num_ranks:
+        raise ValueError("num_ranks must divide H")
+    if not (0.0 <= alpha <= 1.0):
+        raise ValueError("need 0 <= alpha <= 1")
+    hpr = H // num_ranks
+    W = [int(head_work[:, r * hpr:(r + 1) * hpr].sum()) for r in range(num_ranks)]
+    Wstar = max(W)
+    out = np.array(prefix, dtype=np.int64)
+    for r in range(num_ranks):
+        budget = int(math.floor(alpha * float(Wstar - W[r])))
+        n_rows = B * hpr * Nb
+        q, rem = divmod(budget, n_rows)
+        pos = 0
+        for b in range(B):
+            for h in range(r * hpr, (r + 1) * hpr):
+                for i in range(Nb):
+                    share = q + (1 if pos < rem else 0)
+                    out[b, h, i] = min(Nb, int(prefix[b, h, i]) + share)
+                    pos += 1
+    return out
+
+
+def sasa_augment(L: np.ndarray, prefix: np.ndarray, head_work: np.ndarray, num_ranks: int,
+                 alpha: float) -> RepairResult:
+    """Augmented lists: row (b, h, i) keeps the first sasa_extend(...) blocks of its ranking
+    (logits L [B, H, Nb, Nb], descending, ties to the lower id) and its diagonal block."""
+    B, H, Nb = prefix.shape
+    newlen = sasa_extend(prefix, head_work, num_ranks, alpha)
+    mask = np.zeros((B, H, Nb, Nb), dtype=np.uint8)
+    for b in range(B):
+        for h in range(H):
+            for i in range(Nb):
+                mask[b, h, i, rank_order(L[b, h, i])[:newlen[b, h, i]]] = 1
+                mask[b, h, i, i] = 1
+    counts = mask.sum(-1).astype(np.int32)
+    idx = np.full((B, H, Nb, Nb), -1, dtype=np.int32)
+    for b in range(B):
+        for h in range(H):
+            for i in range(Nb):
+                nz = np.nonzero(mask[b, h, i])[0]
+                idx[b, h, i, :nz.size] = nz
+    hw = counts.sum(-1).astype(np.int64)
+    return RepairResult(mask, counts, idx, hw, lpt_worklist(counts))
+
+
 def attention_items(qr_bits, kr_bits, vr_bits, counts, idx, S: int, items: Iterable, scale: Optional[float] = None):
     """Exact float64 output rows of the given items.
 

@@ -401,3 +401,58 @@ def test_reorder_with_hilbert_numbering():
         want = [((bt * g.tt + lt) * g.Y + by * g.ty + ly) * g.X + bx * g.tx + lx
                 for lt in range(g.tt) for ly in range(g.ty) for lx in range(g.tx)]
         assert src[b * g.S:(b + 1) * g.S].tolist() == want
+
+
+# ----------------------------------------------------------------- slack-aware augmentation
+def _routed(cfg):
+    og = O.Geometry.of(cfg)
+    q, k, _ = synth.make_qkv(cfg)
+    rr = O.route(O.reorder(q, og), O.reorder(k, og), og, cfg.p, cfg.k)
+    rp = O.repair(rr.topp_mask, rr.topk_idx)
+    prefix = np.maximum(rr.n_p, min(cfg.k, og.Nb))
+    return og, rr, rp, prefix
+
+
+def test_sasa_hand_case():
+    # B = 1, H = 4 heads of Nb = 2 rows, every row keeping a ranked prefix of 1 block
+    prefix = np.ones((1, 4, 2), dtype=np.int64)
+    hw = np.array([[4, 3, 2, 1]])
+    # 2 ranks {0, 1}, {2, 3}: W = 7, 3, W* = 7; alpha 0.5: B_1 = floor(0.5 * 4) = 2 over the
+    # 4 rows of rank 1 in item order: q = 0, rem = 2, so rows (h2, i0), (h2, i1) get +1
+    assert O.sasa_extend(prefix, hw, 2, 0.5).tolist() == [[[1, 1], [1, 1], [2, 2], [1, 1]]]
+    # alpha 1: B_1 = 4: q = 1 for every row of rank 1
+    assert O.sasa_extend(prefix, hw, 2, 1.0).tolist() == [[[1, 1], [1, 1], [2, 2], [2, 2]]]
+    # 4 ranks, alpha 1: W* = 4, budgets 0, 1, 2, 3 over 2 rows each: (h1, i0) +1; h2 +1, +1;
+    # h3 +2 (capped at Nb = 2), +1
+    assert O.sasa_extend(prefix, hw, 4, 1.0).tolist() == [[[1, 1], [2, 1], [2, 2], [2, 2]]]
+    assert O.sasa_extend(prefix, hw, 4, 0.0).tolist() == prefix.tolist()
+
+
+def test_sasa_invariants():
+    cfg = synth.Config("sasa", B=1, H=4, d=64, T=4, Y=16, X=16, tt=1, ty=8, tx=8, p=0.9, k=2,
+                       a_mode="alternating", a_lo=4.0, a_hi=0.5, noise_std=1.0, sigma=0.3, seed=3)
+    og, rr, rp, prefix = _routed(cfg)
+    for R in (1, 2, 4):
+        for alpha in (0.0, 0.3, 1.0):
+            au = O.sasa_augment(rr.L, prefix, rp.head_work, R, alpha)
+            hpr = cfg.H // R
+            W = [int(rp.head_work[:, r * hpr:(r + 1) * hpr].sum()) for r in range(R)]
+            Wa = [int(au.head_work[:, r * hpr:(r + 1) * hpr].sum()) for r in range(R)]
+            Ws = max(W)
+            assert max(Wa) == Ws                                  # the critical path does not grow
+            for r in range(R):
+                assert Wa[r] - W[r] <= math.floor(alpha * (Ws - W[r]))   # within the rank's budget
+                if W[r] == Ws:
+                    assert Wa[r] == W[r]
+            assert (au.mask >= rp.mask).all()                    # only additions
+            if alpha == 0.0:
+                assert np.array_equal(au.counts, rp.counts)
+            for h in range(cfg.H):                               # kept minus diagonal = a ranked prefix
+                for i in range(og.Nb):
+                    order = O.rank_order(rr.L[0, h, i])
+                    kept = au.mask[0, h, i].copy()
+                    n = int(kept[order].cumprod().sum())
+                    rest = kept.copy()
+                    rest[order[:n]] = 0
+                    rest[i] = 0
+                    assert not rest.any()
