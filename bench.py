@@ -50,7 +50,7 @@ def parse():
     ap.add_argument("--tile-order", choices=("raster", "hilbert"), default="raster",
                     help="tile numbering: raster, or along the 3D Hilbert curve")
     ap.add_argument("--static-order", action="store_true", help="item-id order instead of the LPT work list")
-    ap.add_argument("--report", choices=["stress", "sweep"], default=None,
+    ap.add_argument("--report", choices=["stress", "sweep", "sasa"], default=None,
                     help="instead of the headline line: head-heterogeneity stress (LPT vs item-id order) or the "
                          "p x tile sweep at 720p scale, one JSON line per measurement")
     return ap.parse_args()
@@ -431,9 +431,52 @@ def cta_imbalance(counts, order, n_cta):
     return float(per.max() / per.mean())
 
 
+def run_sasa_report(args):
+    """Slack-aware augmentation at 480p: 8 virtual ranks of 5 heads, alpha 0 .. 1."""
+    import torch
+    import block_sparse_attention_44_b200 as fva
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream(dev)
+    cfg = synth.CONFIGS["wan480p"]
+    g = fva.Geom.of(cfg)
+    q, k, v = synth.make_qkv(cfg)
+    def to_dev(a):
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+    qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
+    path = fva.SparseAttention(g, cfg.p, cfg.k, device=dev)
+    out = torch.empty_like(qd)
+    path(qd, kd, vd, out, stream)
+    ws = torch.empty((fva.fva_sasa_workspace_size(g),), dtype=torch.uint8, device=dev)
+    ranks = 8
+    hpr = g.H // ranks
+    base_hw = path.rep.head_work.clone()
+    W0 = [int(base_hw[:, r * hpr:(r + 1) * hpr].sum()) for r in range(ranks)]
+    for alpha in (0.0, 0.25, 0.5, 1.0):
+        run = lambda: fva.fva_route_repair_sasa(path.qbar, path.kbar, g, cfg.p, cfg.k, ranks, alpha, path.rep.counts,
+                                                path.rep.idx, path.rep.head_work, path.rep.worklist, ws,
+                                                stream=stream)
+        route_ms = _time_ms(run, stream, 5)
+        torch.cuda.synchronize()
+        assert fva.fva_get_device_error(stream) == 0
+        pairs = int(path.rep.counts.sum().item())
+        W1 = [int(path.rep.head_work[:, r * hpr:(r + 1) * hpr].sum()) for r in range(ranks)]
+        attn_ms = _time_ms(lambda: path.attention_natural(out, stream), stream, 3)
+        line = {"report": "sasa", "workload": cfg.name, "virtual_ranks": ranks, "alpha": alpha,
+                "density": pairs / float(g.B * g.H * g.Nb * g.Nb), "pairs_added": pairs - sum(W0),
+                "rank_work_max_over_mean_before": max(W0) / (sum(W0) / ranks),
+                "rank_work_max_over_mean_after": max(W1) / (sum(W1) / ranks),
+                "critical_rank_work": [max(W0), max(W1)],
+                "route_sasa_ms": route_ms, "attn_ms": attn_ms,
+                "attn_tflops": 4.0 * g.S * g.S * g.d * pairs / (attn_ms * 1e-3) / 1e12}
+        print(json.dumps(line), flush=True)
+
+
 def run_report(args):
     import torch
     import block_sparse_attention_44_b200 as fva
+    if args.report == "sasa":
+        run_sasa_report(args)
+        return
     dev = torch.device("cuda", 0)
     stream = torch.cuda.current_stream(dev)
     n_sm = torch.cuda.get_device_properties(dev).multi_processor_count

@@ -97,6 +97,8 @@ def _load():
         "fva_route_static": ([vp, vp, _Geom, f64, i32, vp, vp, vp, vp], ctypes.c_int),
         "fva_route_repair": ([vp, vp, _Geom, f64, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
         "fva_reorder_pool": ([vp, vp, vp, _Geom, vp], ctypes.c_int),
+        "fva_sasa_workspace_size": ([_Geom], sz),
+        "fva_route_repair_sasa": ([vp, vp, _Geom, f64, i32, i32, f64, vp, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
         "fva_route_repair_pooled": ([vp, vp, _Geom, f64, i32, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
         "fva_repair_workspace_size": ([_Geom], sz),
         "fva_repair": ([vp, vp, _Geom, i32, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
@@ -253,6 +255,26 @@ def fva_route_repair_pooled(qbar, kbar, g: Geom, p: float, k: int, counts, idx, 
     _check(lib.fva_route_repair_pooled(_ptr(qbar), _ptr(kbar), g.c(), float(p), int(k), _ptr(topp_mask),
                                        _ptr(topk_idx), _ptr(counts), _ptr(idx), _ptr(head_work), _ptr(worklist),
                                        _stream(stream)))
+
+
+def fva_sasa_workspace_size(g: Geom) -> int:
+    return int(lib.fva_sasa_workspace_size(g.c()))
+
+
+def fva_route_repair_sasa(qbar, kbar, g: Geom, p: float, k: int, num_ranks: int, alpha: float, counts, idx,
+                          head_work, worklist, workspace, extra=None, stream=None):
+    """fva_route_repair_pooled with slack-aware augmentation over num_ranks virtual ranks."""
+    _need(qbar, torch.float64, (g.B, g.H, g.Nb, g.d), "qbar")
+    _need(kbar, torch.float64, (g.B, g.H, g.Nb, g.d), "kbar")
+    _need(counts, torch.int32, (g.B, g.H, g.Nb), "counts")
+    _need(idx, torch.int32, (g.B, g.H, g.Nb, g.Nb), "idx")
+    _need(head_work, torch.int64, (g.B, g.H), "head_work")
+    _need(worklist, torch.int32, (g.B * g.H * g.Nb,), "worklist")
+    if extra is not None:
+        _need(extra, torch.int32, (g.B, g.H, g.Nb), "extra")
+    _check(lib.fva_route_repair_sasa(_ptr(qbar), _ptr(kbar), g.c(), float(p), int(k), int(num_ranks), float(alpha),
+                                     _ptr(counts), _ptr(idx), _ptr(head_work), _ptr(worklist), _ptr(extra),
+                                     _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
 def fva_repair_workspace_size(g: Geom) -> int:

@@ -120,7 +120,7 @@ int finish(cudaError_t e, int launches, const char* where) {
 
 extern "C" {
 
-int32_t fva_version(void) { return 104; }
+int32_t fva_version(void) { return 105; }
 
 const char* fva_last_error(void) { return g_err; }
 
@@ -266,6 +266,42 @@ int fva_route_repair_pooled(const double* qbar, const double* kbar, fva_geom g, 
                                             &launches);
   if (e == cudaSuccess) e = fva::launch_lpt(counts, D, head_work, worklist, s, &launches);
   return finish(e, launches, "fva_route_repair_pooled");
+}
+
+size_t fva_sasa_workspace_size(fva_geom g) {
+  fva::Dims D;
+  if (check_geom(g, D, false)) return 0;
+  return fva::sasa_workspace_bytes(D);
+}
+
+int fva_route_repair_sasa(const double* qbar, const double* kbar, fva_geom g, double p, int32_t k, int32_t num_ranks,
+                          double alpha, int32_t* counts, int32_t* idx, int64_t* head_work, int32_t* worklist,
+                          int32_t* extra, void* workspace, size_t workspace_bytes, void* stream) {
+  fva::Dims D;
+  int rc = check_geom(g, D, false);
+  if (rc) return rc;
+  if (!qbar || !kbar || !counts || !idx || !head_work || !worklist || !workspace)
+    return fail(FVA_ERR_INVALID_ARG, "null pointer");
+  if (!(p > 0.0) || !(p <= 1.0)) return fail(FVA_ERR_INVALID_ARG, "p must satisfy 0 < p <= 1 (got %g)", p);
+  if (k < 1) return fail(FVA_ERR_INVALID_ARG, "k must be >= 1 (got %d)", k);
+  if (num_ranks < 1 || num_ranks > fva::kMaxVirtualRanks || g.H % num_ranks != 0)
+    return fail(FVA_ERR_INVALID_ARG, "num_ranks must divide H and lie in [1, %d] (got %d)", fva::kMaxVirtualRanks,
+                num_ranks);
+  if (!(alpha >= 0.0) || !(alpha <= 1.0)) return fail(FVA_ERR_INVALID_ARG, "alpha must lie in [0, 1] (got %g)", alpha);
+  if (D.Nb > fva::kMaxNb) return fail(FVA_ERR_UNSUPPORTED, "Nb = %d blocks exceeds %d", D.Nb, fva::kMaxNb);
+  if (!aligned16(qbar) || !aligned16(kbar)) return fail(FVA_ERR_INVALID_ARG, "qbar and kbar must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(FVA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  const size_t need = fva::sasa_workspace_bytes(D);
+  if (workspace_bytes < need)
+    return fail(FVA_ERR_INVALID_ARG, "workspace too small: %zu bytes given, %zu needed", workspace_bytes, need);
+  const int kk = k < D.Nb ? k : D.Nb;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int launches = 0;
+  cudaError_t e = fva::launch_sasa(qbar, kbar, D, p, kk, num_ranks, alpha, counts, idx, extra, workspace, s,
+                                   &launches);
+  if (e == cudaSuccess) e = fva::launch_lpt(counts, D, head_work, worklist, s, &launches);
+  return finish(e, launches, "fva_route_repair_sasa");
 }
 
 size_t fva_repair_workspace_size(fva_geom g) {

@@ -44,6 +44,14 @@ cudaError_t launch_repair(const uint8_t* topp_mask, const int32_t* topk_idx, con
                           int32_t* idx, int64_t* head_work, int32_t* worklist, int* dev_err, cudaStream_t s,
                           int* launches);
 
+// Slack-aware augmentation from block means: selection (recording each row's ranked
+// prefix), per-row floors from the virtual-rank budgets, selection again with them.
+cudaError_t launch_sasa(const double* qbar, const double* kbar, const Dims& D, double p, int kk, int num_ranks,
+                        double alpha, int32_t* counts, int32_t* idx, int32_t* extra, void* ws, cudaStream_t s,
+                        int* launches);
+size_t sasa_workspace_bytes(const Dims& D);
+constexpr int kMaxVirtualRanks = 1024;
+
 // Per-head work W_h and the LPT work list from the per-row counts.
 cudaError_t launch_lpt(const int32_t* counts, const Dims& D, int64_t* head_work, int32_t* worklist, cudaStream_t s,
                        int* launches);

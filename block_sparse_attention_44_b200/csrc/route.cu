@@ -38,6 +38,8 @@
 #include <limits.h>
 #include <math.h>
 
+#include <algorithm>
+
 #include "fva_common.cuh"
 #include "fva_internal.h"
 
@@ -60,6 +62,8 @@ struct RouteArgs {
   double* logits_out;   // nullable
   int32_t* counts;      // nullable (no compaction when null)
   int32_t* idx;
+  int32_t* prefix_out;  // nullable: per row, max(n_p, floor) = length of the kept ranked prefix
+  const int32_t* kk_rows;   // nullable: per-row floor replacing kk (topk_idx must then be null)
   int Nb, kk;
   unsigned target;      // ceil(p * 2^31)
   int keep_all_p;       // p >= 1
@@ -266,7 +270,7 @@ __device__ __forceinline__ void select_row(const RouteArgs& a, long long bh, int
   }
 
   // Top-k floor: bit s of `taken` marks block lane + 32 s (kk <= kTopkArgmaxMax)
-  const int kk = a.kk;
+  const int kk = a.kk_rows ? a.kk_rows[row] : a.kk;
   unsigned long long taken = 0;
   unsigned qk = 0;
   u64 kkb = 0;
@@ -352,6 +356,14 @@ __device__ __forceinline__ void select_row(const RouteArgs& a, long long bh, int
     if (!all_p && q[s] == qp) in = at_or_before(Kr[t], t, kpb, jpb);
     if (in && t < Nb) inp |= 1ull << s;
     if (big_k && t < Nb && (q[s] < qk || (q[s] == qk && at_or_before(Kr[t], t, kkb, jkb)))) ink |= 1ull << s;
+  }
+
+  if (a.prefix_out) {   // n_p = size of the Top-p set
+    unsigned np_lane = 0;
+#pragma unroll
+    for (int s = 0; s < PL; ++s) np_lane += static_cast<unsigned>((inp >> s) & 1ull);
+    const int n_p = static_cast<int>(__reduce_add_sync(kFull, np_lane));
+    if (lane == 0) a.prefix_out[row] = n_p > kk ? n_p : kk;
   }
 
   // outputs: compacted kept list, Top-p mask, floor ids (large floors), logits
@@ -547,12 +559,62 @@ RouteArgs make_args(const double* qbar, const double* kbar, const Dims& D, doubl
   a.logits_out = logits_out;
   a.counts = counts;
   a.idx = idx;
+  a.prefix_out = nullptr;
+  a.kk_rows = nullptr;
   a.Nb = D.Nb;
   a.kk = kk;
   a.keep_all_p = p >= 1.0 ? 1 : 0;
   const double tp = ceil(p * 0x1p31);
   a.target = a.keep_all_p ? 0u : static_cast<unsigned>(tp < 1.0 ? 1.0 : tp);
   return a;
+}
+
+// Slack-aware augmentation, single-GPU reading (§3.3 SASA): the heads form num_ranks
+// virtual ranks of H / num_ranks consecutive heads; W_r = kept block pairs of the rank
+// (from the counts); rank r gets B_r = floor(alpha * (W* - W_r)) more pairs, W* the
+// largest W_r, spread round-robin over its rows in item order; a row's floor becomes
+// min(Nb, prefix + share), i.e. its ranked prefix grows by its share.
+constexpr int kSasaThreads = 256;
+constexpr int kSasaMaxRanks = 1024;
+
+__global__ void __launch_bounds__(kSasaThreads) sasa_kernel(const int32_t* __restrict__ counts,
+                                                            const int32_t* __restrict__ prefix, int B, int H, int Nb,
+                                                            int num_ranks, double alpha, int32_t* __restrict__ kk_rows,
+                                                            int32_t* __restrict__ extra) {
+  __shared__ unsigned long long W[kSasaMaxRanks];
+  __shared__ long long budget[kSasaMaxRanks];
+  const int hpr = H / num_ranks;
+  for (int r = threadIdx.x; r < num_ranks; r += kSasaThreads) W[r] = 0;
+  __syncthreads();
+  const long long n = static_cast<long long>(B) * H * Nb;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (long long bh = warp; bh < static_cast<long long>(B) * H; bh += kSasaThreads / 32) {   // W_h, a warp each
+    unsigned long long w = 0;
+    for (int i = lane; i < Nb; i += 32) w += static_cast<unsigned long long>(counts[bh * Nb + i]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) w += __shfl_xor_sync(kFull, w, o);
+    if (lane == 0) atomicAdd(&W[static_cast<int>(bh % H) / hpr], w);
+  }
+  __syncthreads();
+  unsigned long long wmax = 0;
+  for (int r = 0; r < num_ranks; ++r) wmax = W[r] > wmax ? W[r] : wmax;
+  for (int r = threadIdx.x; r < num_ranks; r += kSasaThreads)
+    budget[r] = static_cast<long long>(floor(alpha * static_cast<double>(wmax - W[r])));
+  __syncthreads();
+  const long long n_rows = static_cast<long long>(B) * hpr * Nb;   // rows per rank
+  for (long long u = static_cast<long long>(blockIdx.x) * kSasaThreads + threadIdx.x; u < n;
+       u += static_cast<long long>(gridDim.x) * kSasaThreads) {
+    const int i = static_cast<int>(u % Nb);
+    const int h = static_cast<int>((u / Nb) % H);
+    const long long b = u / (static_cast<long long>(H) * Nb);
+    const int r = h / hpr;
+    const long long pos = (b * hpr + (h - r * hpr)) * Nb + i;        // rank of the row in item order
+    const long long share = budget[r] / n_rows + (pos < budget[r] % n_rows ? 1 : 0);
+    const long long len = prefix[u] + share;
+    const int32_t v = static_cast<int32_t>(len < Nb ? len : Nb);
+    kk_rows[u] = v;
+    if (extra) extra[u] = v - prefix[u];
+  }
 }
 }  // namespace
 
@@ -564,6 +626,29 @@ cudaError_t launch_select_pooled(const double* qbar, const double* kbar, const D
   ++*launches;
   return e;
 }
+
+cudaError_t launch_sasa(const double* qbar, const double* kbar, const Dims& D, double p, int kk, int num_ranks,
+                        double alpha, int32_t* counts, int32_t* idx, int32_t* extra, void* ws, cudaStream_t s,
+                        int* launches) {
+  int32_t* prefix = static_cast<int32_t*>(ws);
+  int32_t* kk_rows = prefix + ((D.rows() + 63) / 64) * 64;
+  RouteArgs a = make_args(qbar, kbar, D, p, kk, nullptr, nullptr, nullptr, counts, idx);
+  a.prefix_out = prefix;
+  cudaError_t e = D.d == 128 ? launch_select<128>(a, 0, D.BH(), s) : launch_select<64>(a, 0, D.BH(), s);
+  ++*launches;
+  if (e != cudaSuccess) return e;
+  const unsigned grid = static_cast<unsigned>(std::min<long long>((D.rows() + kSasaThreads - 1) / kSasaThreads, 148));
+  sasa_kernel<<<grid, kSasaThreads, 0, s>>>(counts, prefix, D.B, D.H, D.Nb, num_ranks, alpha, kk_rows, extra);
+  ++*launches;
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  RouteArgs a2 = make_args(qbar, kbar, D, p, kk, nullptr, nullptr, nullptr, counts, idx);
+  a2.kk_rows = kk_rows;
+  e = D.d == 128 ? launch_select<128>(a2, 0, D.BH(), s) : launch_select<64>(a2, 0, D.BH(), s);
+  ++*launches;
+  return e;
+}
+
+size_t sasa_workspace_bytes(const Dims& D) { return 2 * static_cast<size_t>((D.rows() + 63) / 64) * 64 * sizeof(int32_t); }
 
 cudaError_t launch_route(const void* qr, const void* kr, const Dims& D, double p, int kk, uint8_t* topp_mask,
                          int32_t* topk_idx, double* logits_out, int32_t* counts, int32_t* idx, void* ws,

@@ -12,6 +12,7 @@
  *   fva_route_repair     the two above, fused
  *   fva_reorder_pool, fva_route_repair_pooled
  *                        the same with the pooling done by the reorder pass
+ *   fva_route_repair_sasa  with slack-aware augmentation of the lists
  *   fva_block_sparse_attn  flash-style attention over the kept block pairs
  *   fva_inverse_reorder  back to natural token order
  *   fva_block_sparse_attn_natural  attention with the inverse reorder fused
@@ -182,6 +183,27 @@ int fva_route_repair(const void* qr, const void* kr, fva_geom g, double p, int32
 int fva_route_repair_pooled(const double* qbar, const double* kbar, fva_geom g, double p, int32_t k,
                             uint8_t* topp_mask, int32_t* topk_idx, int32_t* counts, int32_t* idx,
                             int64_t* head_work, int32_t* worklist, void* stream);
+
+/*
+ * fva_route_repair_sasa — fva_route_repair_pooled with slack-aware augmentation, a
+ * single-GPU reading of §3.3 (SASA): the heads form num_ranks virtual ranks of
+ * H / num_ranks consecutive heads (the head layout of Ulysses sequence parallelism,
+ * §2); W_r = kept block pairs of rank r after routing and repair, W* = max_r W_r (the
+ * critical path); rank r receives B_r = floor(alpha * (W* - W_r)) extra block pairs,
+ * spread round-robin over its rows in item order; a row's ranked prefix (the Top-p set
+ * with the floor, following the routing's importance order) grows by its share, capped
+ * at Nb, so no rank's workload passes W* and p is unchanged.  Same outputs as
+ * fva_route_repair_pooled, computed on the augmented lists.
+ *   num_ranks : divides H, 1..1024.     alpha : 0..1 (0: no augmentation).
+ *   extra     : optional int32 [B,H,Nb] output, the ranked positions added to each row.
+ *   workspace : fva_sasa_workspace_size(g) bytes, 256-byte aligned.
+ * Four launches: selection, budgets, selection with the extended floors, LPT list.
+ */
+size_t fva_sasa_workspace_size(fva_geom g);
+int fva_route_repair_sasa(const double* qbar, const double* kbar, fva_geom g, double p, int32_t k,
+                          int32_t num_ranks, double alpha, int32_t* counts, int32_t* idx,
+                          int64_t* head_work, int32_t* worklist, int32_t* extra,
+                          void* workspace, size_t workspace_bytes, void* stream);
 
 /* Workspace bytes fva_repair needs (currently 0; kept for ABI stability). */
 size_t fva_repair_workspace_size(fva_geom g);

@@ -100,6 +100,15 @@ def test_invalid_arguments_rejected_on_host():
         fva.FVA_ERR_INVALID_ARG
     assert L.fva_route_repair_pooled(264, 512, g, 0.9, 1, None, None, 16, 32, 64, 128, None) == \
         fva.FVA_ERR_INVALID_ARG                                                           # qbar misaligned
+    # slack-aware augmentation: num_ranks must divide H, alpha in [0, 1], workspace size
+    sneed = fva.fva_sasa_workspace_size(_g())
+    sargs = lambda R, a, wsb: (256, 512, g, 0.9, 1, R, a, 16, 32, 64, 128, None, 4096, wsb, None)
+    assert L.fva_route_repair_sasa(*sargs(3, 0.5, sneed)) == fva.FVA_ERR_INVALID_ARG     # H = 2
+    assert L.fva_route_repair_sasa(*sargs(0, 0.5, sneed)) == fva.FVA_ERR_INVALID_ARG
+    assert L.fva_route_repair_sasa(*sargs(2, 1.5, sneed)) == fva.FVA_ERR_INVALID_ARG
+    assert L.fva_route_repair_sasa(*sargs(2, float("nan"), sneed)) == fva.FVA_ERR_INVALID_ARG
+    assert L.fva_route_repair_sasa(*sargs(2, 0.5, sneed - 1)) == fva.FVA_ERR_INVALID_ARG
+    assert sneed >= 2 * 4 * _g().B * _g().H * _g().Nb
     # repair / attention: null pointers, k, unsupported tile for attention
     assert L.fva_repair(None, 16, g, 1, 16, 16, 16, 16, None, 0, None) == fva.FVA_ERR_INVALID_ARG
     assert L.fva_repair(16, 16, g, 0, 16, 16, 16, 16, None, 0, None) == fva.FVA_ERR_INVALID_ARG

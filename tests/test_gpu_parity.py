@@ -188,6 +188,62 @@ def test_bad_tile_numbering_entry_is_reported(fva):
     assert fva.fva_get_device_error() == 0
 
 
+@pytest.mark.parametrize("ranks,alpha", [(2, 0.5), (4, 1.0), (1, 1.0), (2, 0.0)])
+def test_sasa_matches_oracle(fva, ranks, alpha):
+    cfg = CASES["stress_small"]                        # alternating sharp / diffuse heads
+    g = fva.Geom.of(cfg)
+    og = O.Geometry.of(cfg)
+    q, k, _ = synth.make_qkv(cfg)
+    shp = (g.B, g.H, g.N, g.d)
+    qr, kr = (torch.empty(shp, dtype=torch.bfloat16, device="cuda") for _ in range(2))
+    qbar, kbar = (torch.empty((g.B, g.H, g.Nb, g.d), dtype=torch.float64, device="cuda") for _ in range(2))
+    fva.fva_reorder_pool(to_dev(q), qr, qbar, g)
+    fva.fva_reorder_pool(to_dev(k), kr, kbar, g)
+    mk = lambda: (torch.empty((g.B, g.H, g.Nb), dtype=torch.int32, device="cuda"),
+                  torch.full((g.B, g.H, g.Nb, g.Nb), -1, dtype=torch.int32, device="cuda"),
+                  torch.empty((g.B, g.H), dtype=torch.int64, device="cuda"),
+                  torch.empty((g.B * g.H * g.Nb,), dtype=torch.int32, device="cuda"))
+    c0, i0, h0, w0 = mk()
+    fva.fva_route_repair_pooled(qbar, kbar, g, cfg.p, cfg.k, c0, i0, h0, w0)
+    c1, i1, h1, w1 = mk()
+    extra = torch.empty((g.B, g.H, g.Nb), dtype=torch.int32, device="cuda")
+    ws = torch.empty((fva.fva_sasa_workspace_size(g),), dtype=torch.uint8, device="cuda")
+    fva.fva_route_repair_sasa(qbar, kbar, g, cfg.p, cfg.k, ranks, alpha, c1, i1, h1, w1, ws, extra=extra)
+    torch.cuda.synchronize()
+    assert fva.fva_get_device_error() == 0
+    rows = g.B * g.H * g.Nb
+    pad = (rows + 63) // 64 * 64
+    wsi = ws.view(torch.int32).cpu().numpy()
+    prefix = wsi[:rows].reshape(g.B, g.H, g.Nb)
+    floors = wsi[pad:pad + rows].reshape(g.B, g.H, g.Nb)
+    # the budget arithmetic is integer work: exact
+    want_len = O.sasa_extend(prefix, h0.cpu().numpy(), ranks, alpha)
+    assert np.array_equal(floors, want_len)
+    assert np.array_equal(extra.cpu().numpy(), want_len - prefix)
+    # the prefixes are the routing's (max(n_p, kk)) outside tie rows
+    rr = O.route(O.reorder(q, og), O.reorder(k, og), og, cfg.p, cfg.k)
+    t1, t2p, t2k = O.tie_flags(rr)
+    ties = t1 | t2p | t2k
+    oracle_prefix = np.maximum(rr.n_p, min(cfg.k, og.Nb))
+    assert np.array_equal(prefix[~ties], oracle_prefix[~ties])
+    # augmented lists: the first floors ranked blocks plus the diagonal, outside tie rows
+    au = O.sasa_augment(rr.L, prefix, h0.cpu().numpy(), ranks, alpha)
+    cnt = c1.cpu().numpy()
+    idx = i1.cpu().numpy()
+    assert np.array_equal(cnt[~ties], au.counts[~ties])
+    valid = np.arange(g.Nb)[None, None, None, :] < cnt[..., None]
+    assert np.array_equal(np.where(valid, idx, -1)[~ties], au.idx[~ties])
+    assert np.array_equal(h1.cpu().numpy(), cnt.sum(-1))
+    assert np.array_equal(w1.cpu().numpy(), O.lpt_worklist(cnt))
+    # the critical path is untouched: no virtual rank ends above the largest one before
+    hpr = g.H // ranks
+    W0 = [int(h0[:, r * hpr:(r + 1) * hpr].sum()) for r in range(ranks)]
+    W1 = [int(h1[:, r * hpr:(r + 1) * hpr].sum()) for r in range(ranks)]
+    assert max(W1) == max(W0)
+    if alpha == 0.0:
+        assert torch.equal(c1, c0)
+
+
 def test_lpt_and_static_order_identical(fva):
     cfg = CASES["d128_s128_multiwave"]
     g = fva.Geom.of(cfg)
