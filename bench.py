@@ -1,13 +1,16 @@
 """Benchmark of the adaptive block-sparse attention path on B200.
 
 One step = one pass of the whole path over one Wan-like attention layer held in
-HBM: reorder(Q, K, V) -> route -> repair -> block-sparse attention -> inverse
-reorder.  `value` is the step's throughput in actual (sparse) attention TFLOP/s;
-the JSON line also carries the dense-equivalent rate, the routing GB/s, the
-attention kernel's roofline fraction, an end-to-end figure through host buffers,
-the clocks seen while timing, and the CPU oracle timed on a bounded sample.
+HBM: reorder(Q, K with pooling; V) -> route + repair from the pooled means ->
+block-sparse attention writing the output in natural order (6 launches).  `value`
+is the step's throughput in actual (sparse) attention TFLOP/s; the JSON line also
+carries the dense-equivalent rate, the routing GB/s (standalone and together with
+the reorder), the attention kernel's roofline fraction, an end-to-end figure through
+host buffers, the clocks seen while timing, and the CPU oracle timed on a bounded
+sample.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config wan480p] [--impl reference]
+                    [--tile-order raster|hilbert] [--static-order] [--report stress|sweep|sasa]
 
 Multi-GPU (torchrun): every rank runs its own replica of the layer (weak scaling,
 no data-path collective); the time is the max over ranks.
