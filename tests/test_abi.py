@@ -146,3 +146,31 @@ def test_tile_order_table_matches_oracle():
     bad = _g().c()
     bad.tile_order = 18                                   # not 4-byte aligned
     assert fva.lib.fva_reorder(16, 32, bad, None) == fva.FVA_ERR_INVALID_ARG
+
+
+def _declarations():
+    """name -> parameter count of every function the header declares."""
+    out = {}
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if not f.endswith(".h"):
+            continue
+        src = re.sub(r"/\*.*?\*/", "", open(os.path.join(ROOT, "include", f)).read(), flags=re.S)
+        for m in re.finditer(r"\b(fva_[a-z0-9_]+)\s*\(([^)]*)\)\s*;", src):
+            params = m.group(2).strip()
+            out[m.group(1)] = 0 if params in ("", "void") else len(params.split(","))
+    return out
+
+
+def test_binding_signatures_match_the_header():
+    decl = _declarations()
+    assert len(decl) >= 15
+    for name, n in decl.items():
+        f = getattr(fva.lib, name)
+        assert f.argtypes is not None, f"{name}: no ctypes signature in the binding"
+        assert len(f.argtypes) == n, f"{name}: header has {n} parameters, binding {len(f.argtypes)}"
+
+
+def test_geometry_struct_layout():
+    # 9 int32 sizes, then the tile-numbering pointer (8-byte aligned)
+    assert ctypes.sizeof(fva._Geom) == 48
+    assert fva._Geom.tile_order.offset == 40
