@@ -17,7 +17,7 @@ import torch
 __all__ = [
     "FvaError", "Geom", "lib", "fva_reorder", "fva_inverse_reorder", "fva_route_workspace_size", "fva_route",
     "fva_route_static", "fva_repair_workspace_size", "fva_repair", "fva_block_sparse_attn", "fva_get_device_error", "fva_last_error",
-    "fva_launch_count", "fva_version", "RouteOutputs", "RepairOutputs", "SparseAttention",
+    "fva_launch_count", "fva_version", "RouteOutputs", "RepairOutputs", "SparseAttention", "HostPipeline",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -427,3 +427,76 @@ class SparseAttention:
             self.attention(stream)
             fva_inverse_reorder(self.outr, out, g, stream)
         return out
+
+
+class HostPipeline:
+    """The whole path over batches held in pinned host memory, with the copies hidden
+    under the kernels: the host->device copy of batch s+1 and the device->host copy of
+    batch s-1 run while batch s computes.
+
+    Two device input sets and two device outputs alternate between batches, on three
+    streams: copy-in, compute (the path's kernels in order) and copy-out.  Only the
+    reorder pass reads an input set (everything after it reads the tile-major copies),
+    so a set may be overwritten once its reorder has run; an output may be overwritten
+    once its copy-out has run.  Events carry exactly those two hazards plus the two
+    data dependencies (copy-in before reorder, attention before copy-out).
+
+    `submit` enqueues one batch and returns an event recorded after its copy-out; the
+    host tensors must stay alive and unmodified until that event completes.
+    """
+
+    def __init__(self, path: SparseAttention, compute_stream=None):
+        g = path.g
+        dev = path.qr.device
+        shp = (g.B, g.H, g.N, g.d)
+        self.path = path
+        self.compute = compute_stream if compute_stream is not None else torch.cuda.current_stream(dev)
+        self.copy_in = torch.cuda.Stream(dev)
+        self.copy_out = torch.cuda.Stream(dev)
+        self.inputs = [tuple(torch.empty(shp, dtype=torch.bfloat16, device=dev) for _ in range(3)) for _ in range(2)]
+        self.outputs = [torch.empty(shp, dtype=torch.bfloat16, device=dev) for _ in range(2)]
+        self.in_free = [None, None]    # reorder of the set's last batch has run
+        self.out_free = [None, None]   # copy-out of the output's last batch has run
+        self.count = 0
+
+    def submit(self, qh: torch.Tensor, kh: torch.Tensor, vh: torch.Tensor, outh: torch.Tensor) -> torch.cuda.Event:
+        j = self.count % 2
+        ins, out = self.inputs[j], self.outputs[j]
+        for h, name in ((qh, "q"), (kh, "k"), (vh, "v"), (outh, "out")):
+            if h.dtype != torch.bfloat16 or tuple(h.shape) != tuple(out.shape):
+                raise ValueError(f"{name}: expected bf16 of shape {tuple(out.shape)}, got {h.dtype} {tuple(h.shape)}")
+            if h.is_cuda or not h.is_pinned() or not h.is_contiguous():
+                raise ValueError(f"{name}: must be a contiguous pinned host tensor")
+        if self.in_free[j] is not None:
+            self.copy_in.wait_event(self.in_free[j])
+        with torch.cuda.stream(self.copy_in):
+            for d, h in zip(ins, (qh, kh, vh)):
+                d.copy_(h, non_blocking=True)
+        in_ready = torch.cuda.Event()
+        in_ready.record(self.copy_in)
+
+        self.compute.wait_event(in_ready)
+        self.path.reorder_qkv(*ins, self.compute)
+        self.in_free[j] = torch.cuda.Event()
+        self.in_free[j].record(self.compute)
+        self.path.routing(self.compute)
+        if self.out_free[j] is not None:
+            self.compute.wait_event(self.out_free[j])
+        self.path.attention_natural(out, self.compute)
+        out_ready = torch.cuda.Event()
+        out_ready.record(self.compute)
+
+        self.copy_out.wait_event(out_ready)
+        with torch.cuda.stream(self.copy_out):
+            outh.copy_(out, non_blocking=True)
+        self.out_free[j] = torch.cuda.Event()
+        self.out_free[j].record(self.copy_out)
+        self.count += 1
+        return self.out_free[j]
+
+    def join(self, stream=None) -> None:
+        """Make `stream` (default: the compute stream) wait for every enqueued copy-out."""
+        s = self.compute if stream is None else stream
+        for e in self.out_free:
+            if e is not None:
+                s.wait_event(e)

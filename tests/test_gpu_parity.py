@@ -334,3 +334,44 @@ def test_out_of_range_block_id_is_reported(fva):
     fva.fva_block_sparse_attn(to_dev(q), to_dev(k), to_dev(v), counts, idx, None, g, 0.0, out)
     assert fva.fva_get_device_error() == 2
     assert fva.fva_get_device_error() == 0         # cleared by the read
+
+
+def test_host_pipeline_matches_per_batch_path(fva):
+    """Three different batches through HostPipeline (copies overlapped with the kernels,
+    device buffers alternating) each give that batch's own device-resident result, bit
+    for bit (that result is held to the oracle by test_path_matches_oracle)."""
+    cfg = CASES["d128_s128_multiwave"]
+    g = fva.Geom.of(cfg)
+    path = fva.SparseAttention(g, cfg.p, cfg.k, device="cuda")
+    pipe = fva.HostPipeline(path)
+    hosts = []
+    for seed in (11, 12, 13):
+        q, k, v = synth.make_qkv(cfg.with_(seed=seed))
+        hosts.append(tuple(torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).pin_memory()
+                           for a in (q, k, v)))
+    outs = [torch.empty(hosts[0][0].shape, dtype=torch.bfloat16).pin_memory() for _ in hosts]
+    for (qh, kh, vh), oh in zip(hosts, outs):
+        pipe.submit(qh, kh, vh, oh)
+    pipe.join()
+    torch.cuda.synchronize()
+    assert fva.fva_get_device_error() == 0
+    for (qh, kh, vh), oh in zip(hosts, outs):
+        ref = torch.empty(qh.shape, dtype=torch.bfloat16, device="cuda")
+        path(qh.cuda(), kh.cuda(), vh.cuda(), ref)
+        torch.cuda.synchronize()
+        assert torch.equal(oh.view(torch.int16), ref.cpu().view(torch.int16))
+    assert not torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
+
+
+def test_host_pipeline_rejects_device_and_pageable_tensors(fva):
+    cfg = CASES["tiny"]
+    g = fva.Geom.of(cfg)
+    pipe = fva.HostPipeline(fva.SparseAttention(g, cfg.p, cfg.k, device="cuda"))
+    shp = (g.B, g.H, g.N, g.d)
+    pinned = torch.zeros(shp, dtype=torch.bfloat16).pin_memory()
+    with pytest.raises(ValueError):
+        pipe.submit(torch.zeros(shp, dtype=torch.bfloat16), pinned, pinned, pinned)
+    with pytest.raises(ValueError):
+        pipe.submit(pinned, pinned, pinned, torch.zeros(shp, dtype=torch.bfloat16, device="cuda"))
+    with pytest.raises(ValueError):
+        pipe.submit(pinned, pinned, pinned, torch.zeros((1,) + shp, dtype=torch.bfloat16).pin_memory())
