@@ -322,6 +322,8 @@ def test_tie_flags_detect_constructed_ties():
     # the cumulative mass lands exactly on p (dyadic masses .5, .25, ...)
     t1, t2p, t2k = _flags_for_row(np.log([0.5, 0.25, 0.125, 0.125]), 0.75, 1)
     assert t1 and not t2p and not t2k
+    # the mass of the ranked prefix one short of the cut lies 1e-7 below p
+    assert _flags_for_row(np.log([0.5, 0.2499999, 0.2, 0.0500001]), 0.75, 1) == [True, False, False]
     # a clean row raises no flag
     assert _flags_for_row([3.0, 1.0, 0.0, -2.0], 0.85, 1) == [False, False, False]
 
@@ -387,6 +389,15 @@ def test_tile_order_raster_is_identity_and_hilbert_a_permutation():
         assert sum(abs(int(x) - int(y)) for x, y in zip(ca, cb)) == 1
 
 
+def test_tile_order_2x2x2_grid_follows_the_hand_derived_curve():
+    # a 2 x 2 x 2 tile grid numbers its tiles along the hand-derived 2x2x2 curve; cell
+    # (bt, by, bx) is raster tile (bt * 2 + by) * 2 + bx
+    fx = json.load(open(os.path.join(GOLDEN, "hilbert_fixture.json")))
+    g = O.Geometry(1, 1, 4, 16, 16, 64, 2, 8, 8, "hilbert")
+    want = [(bt * 2 + by) * 2 + bx for bt, by, bx in fx["cells_in_order"]]
+    assert O.tile_order(g).tolist() == want
+
+
 def test_reorder_with_hilbert_numbering():
     g = O.Geometry(1, 2, 4, 16, 24, 64, 2, 8, 8, "hilbert")       # 2 x 2 x 3 tiles
     x = np.random.default_rng(5).integers(0, 1 << 16, size=(1, 2, g.N, 64), dtype=np.uint16)
@@ -420,6 +431,8 @@ def test_sasa_hand_case():
     # 2 ranks {0, 1}, {2, 3}: W = 7, 3, W* = 7; alpha 0.5: B_1 = floor(0.5 * 4) = 2 over the
     # 4 rows of rank 1 in item order: q = 0, rem = 2, so rows (h2, i0), (h2, i1) get +1
     assert O.sasa_extend(prefix, hw, 2, 0.5).tolist() == [[[1, 1], [1, 1], [2, 2], [1, 1]]]
+    # alpha 0.3: B_1 = floor(1.2) = 1, to the first row of rank 1 only
+    assert O.sasa_extend(prefix, hw, 2, 0.3).tolist() == [[[1, 1], [1, 1], [2, 1], [1, 1]]]
     # alpha 1: B_1 = 4: q = 1 for every row of rank 1
     assert O.sasa_extend(prefix, hw, 2, 1.0).tolist() == [[[1, 1], [1, 1], [2, 2], [2, 2]]]
     # 4 ranks, alpha 1: W* = 4, budgets 0, 1, 2, 3 over 2 rows each: (h1, i0) +1; h2 +1, +1;
