@@ -229,8 +229,11 @@ int fva_repair(const uint8_t* topp_mask, const int32_t* topk_idx, fva_geom g, in
  * overview: block-sparse attention after routing; §2: only selected block pairs
  * are evaluated).  Bidirectional, no causal mask.
  *   qr, kr, vr : bf16 [B,H,N,d] tile-major.
- *   counts,idx : fva_repair outputs (every listed id must be in [0, Nb)).
- *   worklist   : fva_repair's LPT order, or NULL for item-id order.
+ *   counts,idx : fva_repair outputs (every listed id must be in [0, Nb); an id outside
+ *                it sets device error 2 and is replaced by the row's own block i).  A
+ *                count above Nb is read as Nb; a row with count <= 0 gets all-zero output.
+ *   worklist   : fva_repair's LPT order, or NULL for item-id order (an entry outside
+ *                [0, B*H*Nb) sets device error 2 and is skipped).
  *   softmax_scale : <= 0 selects 1/sqrt(d).
  *   out_r      : bf16 [B,H,N,d] tile-major output, O_i = softmax(Q_i K_J^T * scale) V_J
  *                over the union J of the kept key blocks of query block i.
