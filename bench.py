@@ -42,7 +42,7 @@ DEFAULT_CONFIG = "wan480p"
 METRIC = "block-sparse attn TFLOPS (actual & dense-equiv) + % bf16 peak; routing GB/s, 1\u00d7B200"
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
@@ -56,7 +56,7 @@ def parse():
     ap.add_argument("--report", choices=["stress", "sweep", "sasa"], default=None,
                     help="instead of the headline line: head-heterogeneity stress (LPT vs item-id order) or the "
                          "p x tile sweep at 720p scale, one JSON line per measurement")
-    return ap.parse_args()
+    return ap.parse_args(argv)
 
 
 def workload_desc(cfg) -> dict:
@@ -69,6 +69,15 @@ def workload_desc(cfg) -> dict:
                                              f"[{cfg.a_lo}, {cfg.a_hi}], noise std {cfg.noise_std:.3g}, seed {cfg.seed}",
         "l2": f"inputs larger than L2 ({cfg.B * cfg.H * cfg.N * cfg.d * 2 / 1e6:.0f} MB per Q/K/V tensor)",
     }
+
+
+DATA = "synthetic (seeded random-Fourier-feature Q/K, Gaussian V; stands in for Wan2.2 latents)"
+
+
+def arm_config(cfg, args, world: int) -> dict:
+    """The `config` object of the JSON line, the same for the GPU arm and the reference arm."""
+    return dict(workload_desc(cfg), parallelism=f"replicas x{world} (no data-path collective)",
+                order="static" if args.static_order else "lpt", tiles=args.tile_order)
 
 
 def load_peaks() -> dict:
@@ -221,7 +230,7 @@ def run_reference(args, rank: int, world: int):
         "impl": "reference", "metric": METRIC, "value": value,
         "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * statistics.median(secs), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": workload_desc(cfg),
+        "vs_baseline": None, "dtype": "f64", "data": DATA, "config": arm_config(cfg, args, world),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -397,9 +406,8 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "bf16",
-        "data": "synthetic (seeded random-Fourier-feature Q/K, Gaussian V; stands in for Wan2.2 latents)",
-        "config": dict(workload_desc(cfg), parallelism=f"replicas x{world} (no data-path collective)",
-                       order="static" if args.static_order else "lpt", tiles=args.tile_order),
+        "data": DATA,
+        "config": arm_config(cfg, args, world),
         "dense_equiv_tflops": whole_job_rate(world, flops_dense, ms) / 1e12,
         "attn_pct_bf16_peak": 100.0 * achieved / peak,
         "attn_pct_bf16_peak_burst": 100.0 * achieved / peaks["bf16_tflops"],

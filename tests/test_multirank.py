@@ -70,3 +70,15 @@ def test_reference_arm_two_ranks():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+                "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["steps"] == 1 and d["warmup"] == 1 and d["e2e"]["value"] == d["value"]
+    assert d["cpu_baseline"]["value"] == d["value"] and d["cpu_baseline"]["cores"] >= 1
+    # the same metric, unit, direction, data and config object as the GPU arm prints
+    sys.path.insert(0, ROOT)
+    import bench
+    args = bench.parse(["--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "1"])
+    cfg = bench.synth.CONFIGS[args.config]
+    assert d["config"] == json.loads(json.dumps(bench.arm_config(cfg, args, 2)))
+    assert (d["metric"], d["unit"], d["higher_is_better"], d["data"]) == (bench.METRIC, "TFLOP/s", True, bench.DATA)
