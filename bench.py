@@ -6,8 +6,9 @@ block-sparse attention writing the output in natural order (6 launches).  `value
 is the step's throughput in actual (sparse) attention TFLOP/s; the JSON line also
 carries the dense-equivalent rate, the routing GB/s (standalone and together with
 the reorder), the attention kernel's roofline fraction, an end-to-end figure through
-host buffers, the clocks seen while timing, and the CPU oracle timed on a bounded
-sample.
+host buffers (HostPipeline, the copies overlapped with the kernels; the serial
+copy-compute-copy figure beside it), the clocks seen while timing, and the CPU oracle
+timed on a bounded sample.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config wan480p] [--impl reference]
                     [--tile-order raster|hilbert] [--static-order] [--report stress|sweep|sasa]
