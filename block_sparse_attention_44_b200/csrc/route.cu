@@ -20,7 +20,8 @@
 // Selection arithmetic (deterministic, exact integer sums):
 //   - softmax weights e_j = 2^((L_ij - max_j L_ij) log2 e) in float32 (the float64
 //     difference rounded once, then the hardware base-2 exponential), z = sum_j e_j
-//     pairwise in float32, and the mass m_j = floor(e_j * (2^31 / z)) as an integer;
+//     in float32 (per lane, then across the warp), and the mass
+//     m_j = floor(e_j * (2^31 / z)) as an integer;
 //   - the Top-p boundary is the first position, in the ranking (logit descending,
 //     block id ascending), where the running sum of m reaches ceil(p * 2^31): found
 //     by a 14-step bisection over the bucket index q_j = floor((max L - L_ij) * 256)
@@ -29,12 +30,22 @@
 //   - the Top-k floor by repeated warp argmax over (logit, -block id); argmaxes are
 //     three integer warp reductions over an order-preserving key of the float64 logit,
 //     so every ranking decision is exact.
-// Error of the running mass at any cut against the exact cumulative softmax mass:
-// rounding of the exponent argument (|x| <= 65, 2^-24 relative) weighted by the masses
-// <= 5e-7, the exponential (2^-22 relative) 2.4e-7, z (pairwise, 8 levels) 4.8e-7, the
-// scaling 1.2e-7, truncation Nb * 2^-31 <= 1e-6: in all below 2.5e-6.  A kept set can
-// differ from the exact one only where the cumulative mass at the cut lies that close
-// to p (rows the parity rule flags as ties, whose band is 1e-5).
+// Error of the running mass at any cut against the exact cumulative softmax mass C_n
+// (u = 2^-24).  Relative errors eps_j of the weights move the cut's mass by at most
+// sum_j mass_j * eps_j (an error common to the kept and the dropped part cancels):
+//   - the exponent argument x_j = (L_j - max) log2 e rounded to float32: eps_j <=
+//     ln2 |x_j| u, and sum_j mass_j |x_j| <= log2 Nb (an entropy): 4.5e-7 at Nb = 2048;
+//   - the hardware exponential, 2^-22 relative: 2.4e-7.
+// z is summed in float32, sequentially over a lane's PL slots and then across the warp,
+// so at most PL + 4 roundings lie on any path: (PL + 4) u relative, which moves C_n by
+// 7.2e-7 (PL = 8, Nb <= 256), 1.4e-6 (PL = 20, Nb <= 640), 2.6e-6 (PL = 40, Nb <= 1280)
+// or 4.1e-6 (PL = 64, Nb <= 2048).  The scaling 2^31 / z and the product add 2u
+// (1.2e-7); truncating each mass to 2^-31 loses at most Nb * 2^-31 (9.5e-7 at
+// Nb = 2048); weights below e^-45 set to 0 lose less than Nb e^-45 < 1e-16.
+// In all: below 2.5e-6 for Nb <= 640 (the 128-token tiles of the 480p and 720p layers)
+// and below 6e-6 up to Nb = 2048, inside the 1e-5 band of the parity rule's cumulative-
+// mass ties.  A kept set can differ from the exact one only where the cumulative mass
+// at the cut lies that close to p.
 #include <limits.h>
 #include <math.h>
 

@@ -120,11 +120,12 @@ size_t fva_route_workspace_size(fva_geom g);
  *                blocks of each row, in ascending block id.
  *   logits_out : optional float64 [B,H,Nb,Nb] output of Qbar_i.Kbar_j/sqrt(d), or NULL.
  * Arithmetic: per-block means and logits in float64; rows ranked by logit descending,
- * ties to the lower block id.  Softmax masses are the float64 weights exp(L - max L)
+ * ties to the lower block id.  Softmax weights 2^((L - max L) log2 e) in float32,
  * normalised and truncated to 2^-31 fixed point; the running mass is an exact integer
  * sum, so the result is deterministic and the cumulative mass at any cut is within
- * 1.2e-6 of the exact one (a kept set differs from the exact rule only where the
- * cumulative mass at the cut lies that close to p).  Requires Nb <= 2048.
+ * 2.5e-6 of the exact one for Nb <= 640 and within 6e-6 up to Nb = 2048 (a kept set
+ * differs from the exact rule only where the cumulative mass at the cut lies that close
+ * to p).  Requires Nb <= 2048.
  * Two kernel launches on `stream`: pooling, then scoring and selection.
  */
 int fva_route(const void* qr, const void* kr, fva_geom g, double p, int32_t k,
