@@ -235,7 +235,7 @@ __device__ __forceinline__ void select_row(const RouteArgs& a, long long bh, int
   warp_best(order_key(lmax), 0u, mk, mt);
   const double mx = key_value(mk);
 
-  // weights 2^((L - max) log2 e) on the MUFU unit, summed pairwise in float32; blocks
+  // weights 2^((L - max) log2 e) on the MUFU unit, summed in float32 per lane then across the warp; blocks
   // more than 45 below the max (weight < e^-45, mass 0) go to bucket kQCap
   unsigned q[PL], m[PL];
   float zl = 0.0f;
