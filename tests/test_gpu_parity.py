@@ -98,7 +98,14 @@ WIDE = {
     "nb300_d128": _cfg("nb300_d128", H=2, T=3, Y=80, X=80, tt=1, ty=8, tx=8, seed=21),
     "nb700_d64": _cfg("nb700_d64", H=2, d=64, T=7, Y=80, X=80, tt=1, ty=8, tx=8, seed=22),
     "nb1500_d128": _cfg("nb1500_d128", H=1, T=15, Y=80, X=80, tt=1, ty=8, tx=8, p=0.95, k=20, seed=23),
+    # the widest row the selection takes (Nb = 2048: every lane slot used); the Top-p sets
+    # hold 138 to 341 blocks
+    "nb2048_d64": _cfg("nb2048_d64", H=1, d=64, T=8, Y=128, X=128, tt=1, ty=8, tx=8, k=8, a_mode="fixed",
+                       a_lo=4.0, a_hi=4.0, sigma=0.6, seed=24),
 }
+# rows whose cut falls deep in a flat tail climb to p in small steps, so more of them
+# land in the 1e-5 tie band (6 % of the 2048 rows of nb2048_d64 in the oracle)
+WIDE_TIE_FRAC = {"nb2048_d64": 0.1}
 
 
 @pytest.mark.parametrize("name", list(WIDE))
@@ -129,7 +136,7 @@ def test_route_wide_rows(fva, name):
     mask_dev, topk_dev = mask.cpu().numpy(), topk.cpu().numpy()
     # a diffuse row of Nb blocks climbs to p in steps of about 1/Nb of the mass, so the
     # 1e-5 band around p flags about 2e-5 * Nb of such rows (2.4 % at Nb = 700)
-    check_route(rr, mask_dev, topk_dev, max_tie_frac=0.05)
+    check_route(rr, mask_dev, topk_dev, max_tie_frac=WIDE_TIE_FRAC.get(name, 0.05))
     check_repair(dict(counts=counts, idx=idx, head_work=hw, worklist=wl), mask_dev, topk_dev)
 
 
