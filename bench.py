@@ -324,6 +324,8 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
             e[3].record(stream)
         stop.record(stream)
         torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
     launches = fva.fva_launch_count() - launches0
     assert fva.fva_get_device_error(stream) == 0
     total_ms = max_over_ranks(start.elapsed_time(stop), world, dev)
