@@ -107,8 +107,57 @@ def check_pooled(dev: dict, q: np.ndarray, k: np.ndarray, og):
     assert torch.equal(torch.where(valid, res["idx"], -1), torch.where(valid, dev["idx"], -1))
 
 
+TIE_TOL = 1e-5
+
+
+def _near_top_set(L_row: np.ndarray, members: np.ndarray, n: int, tol: float) -> bool:
+    """`members` (bool [Nb], n of them set) is a set of the n highest logits of the row,
+    up to swaps of blocks whose logits lie within tol * max(1, |L|) of the n-th
+    highest: no member lies clearly below it and no non-member clearly above it."""
+    Ls = L_row[O.rank_order(L_row)]
+    thr = Ls[n - 1]
+    band = tol * max(1.0, abs(thr))
+    return not (L_row[members] < thr - band).any() and not (L_row[~members] > thr + band).any()
+
+
+def valid_tie_topp(L_row, P_row, mask_row, p, tol=TIE_TOL) -> bool:
+    """A Top-p set another rounding of the masses may legitimately choose on a tie row:
+    a ranked prefix (up to near-equal logits at its end) whose exact mass reaches
+    p - tol, and which is minimal within tol (dropping its lowest-ranked block leaves
+    less than p + tol).  Keeping every block is valid when the exact total mass lies
+    within tol of p or below it."""
+    members = mask_row.astype(bool)
+    n = int(members.sum())
+    Nb = members.size
+    if n == 0 or not _near_top_set(L_row, members, n, tol):
+        return False
+    mass = float(P_row[members].sum())
+    if n == Nb and float(P_row.sum()) < p + tol:
+        return True
+    if mass < p - tol:
+        return False
+    rank = np.empty(Nb, dtype=np.int64)
+    rank[O.rank_order(L_row)] = np.arange(Nb)
+    idx = np.nonzero(members)[0]
+    last = idx[np.argmax(rank[idx])]
+    return mass - float(P_row[last]) < p + tol
+
+
+def valid_tie_topk(L_row, ids, kk, tol=TIE_TOL) -> bool:
+    """kk distinct ascending block ids forming a set of the kk highest logits, up to
+    swaps among logits within tol * max(1, |L|) at the floor boundary."""
+    ids = np.asarray(ids)
+    if ids.size != kk or (np.diff(ids) <= 0).any() or ids.min() < 0 or ids.max() >= L_row.size:
+        return False
+    members = np.zeros(L_row.size, dtype=bool)
+    members[ids] = True
+    return _near_top_set(L_row, members, kk, tol)
+
+
 def check_route(rr: O.RouteResult, mask_dev: np.ndarray, topk_dev: np.ndarray, max_tie_frac=0.02):
-    """Bit-exact comparison except rows flagged as ties; returns (n_rows, n_tie_rows, n_diff_rows)."""
+    """Bit-exact comparison except rows flagged as ties; a tie row where the device
+    differs must still hold a valid answer (valid_tie_topp / valid_tie_topk).
+    Returns (n_rows, n_tie_rows, n_diff_rows); every differing row was validated."""
     t1, t2p, t2k = O.tie_flags(rr)
     dm = (mask_dev != rr.topp_mask).any(-1)
     dk = (topk_dev != rr.topk_idx).any(-1)
@@ -116,6 +165,13 @@ def check_route(rr: O.RouteResult, mask_dev: np.ndarray, topk_dev: np.ndarray, m
     bad_k = dk & ~t2k
     assert not bad_m.any(), f"{int(bad_m.sum())} Top-p rows differ without a tie, e.g. {np.argwhere(bad_m)[:5]}"
     assert not bad_k.any(), f"{int(bad_k.sum())} Top-k rows differ without a tie, e.g. {np.argwhere(bad_k)[:5]}"
+    kk = rr.topk_idx.shape[-1]
+    for b, h, i in np.argwhere(dm):
+        assert valid_tie_topp(rr.L[b, h, i], rr.P[b, h, i], mask_dev[b, h, i], rr.p), \
+            f"tie row {(b, h, i)}: device Top-p set is not a valid answer"
+    for b, h, i in np.argwhere(dk):
+        assert valid_tie_topk(rr.L[b, h, i], topk_dev[b, h, i], kk), \
+            f"tie row {(b, h, i)}: device floor is not a valid top-{kk} set"
     ties = t1 | t2p | t2k
     assert ties.mean() <= max_tie_frac, f"tie rows {ties.mean():.4f} above {max_tie_frac}"
     return int(ties.size), int(ties.sum()), int((dm | dk).sum())

@@ -124,8 +124,13 @@ def _cut_one_short(C, p, Nb):
     return int(hit[0]) if hit.size else Nb
 
 
-def _route_with(floor_ids):
+def _route_with(floor_ids=lambda order, kk: order[:kk], rows="q", cols="k"):
+    """route() with a planted mistake: the floor taken from elsewhere in the ranking, or
+    the pooled operands wired to the wrong side of the score matrix (rows / cols name
+    the tensor whose block means form Qbar / Kbar)."""
     def f(qr_bits, kr_bits, g, p, k):
+        src = {"q": qr_bits, "k": kr_bits}
+        qr_bits, kr_bits = src[rows], src[cols]
         B, H, Nb = g.B, g.H, g.Nb
         kk = min(k, Nb)
         L = np.empty((B, H, Nb, Nb))
@@ -328,6 +333,9 @@ MUTANTS = [
      [("test_topp_hand_fixtures", ()), ("test_topp_bruteforce_small", (5,)), ("test_floor_and_diagonal_invariants", ())]),
     ("floor-from-the-tail", "route", _route_with(lambda order, kk: order[-kk:]),
      [("test_tiny_p_reduces_to_topk_union_diag", ())]),
+    ("route-operands-swapped", "route", _route_with(rows="k", cols="q"), [("test_route_operand_order_hand_case", ())]),
+    ("route-q-against-q", "route", _route_with(rows="q", cols="q"), [("test_route_operand_order_hand_case", ())]),
+    ("route-k-against-k", "route", _route_with(rows="k", cols="k"), [("test_route_operand_order_hand_case", ())]),
     ("repair-drops-floor", "repair", _repair_with(floor=False),
      [("test_repair_compaction_and_head_work", ()), ("test_tiny_p_reduces_to_topk_union_diag", ())]),
     ("repair-drops-diagonal", "repair", _repair_with(diagonal=False),

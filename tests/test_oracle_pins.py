@@ -193,6 +193,32 @@ def test_topk_ties_prefer_lower_index():
     assert order[:3].tolist() == [0, 1, 2]
 
 
+def _f32_to_bf16_bits(a) -> np.ndarray:
+    """Bit patterns of values that bfloat16 holds exactly (checked)."""
+    f = np.asarray(a, dtype=np.float32)
+    bits = (f.view(np.uint32) >> 16).astype(np.uint16)
+    assert np.array_equal((bits.astype(np.uint32) << 16).view(np.float32), f)
+    return bits
+
+
+def test_route_operand_order_hand_case():
+    """Pooled Q goes to the rows of the score matrix and pooled K to its columns: a
+    hand-derived case with Qbar and Kbar deliberately different (a transposed or
+    self-paired wiring keeps other sets)."""
+    fx = json.load(open(os.path.join(GOLDEN, "route_operand_fixture.json")))
+    gd = fx["geometry"]
+    g = O.Geometry(gd["B"], gd["H"], gd["T"], gd["Y"], gd["X"], gd["d"], gd["tt"], gd["ty"], gd["tx"])
+    q = _f32_to_bf16_bits(fx["q_tokens"])[None]
+    k = _f32_to_bf16_bits(fx["k_tokens"])[None]
+    rr = O.route(O.reorder(q, g), O.reorder(k, g), g, fx["p"], fx["k"])
+    assert np.array_equal(rr.L[0], np.array(fx["L"], dtype=np.float64))
+    assert rr.topp_mask[0].tolist() == fx["topp_mask"]
+    assert rr.n_p[0].tolist() == fx["n_p"]
+    assert rr.topk_idx[0].tolist() == fx["topk_idx"]
+    rp = O.repair(rr.topp_mask, rr.topk_idx)
+    assert rp.counts[0].tolist() == fx["repaired_counts"]
+
+
 # ---------------------------------------------------------------- repair / LPT ----
 def test_repair_compaction_and_head_work():
     rng = np.random.default_rng(8)
