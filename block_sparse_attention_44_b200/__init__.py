@@ -99,12 +99,13 @@ def _load():
         "fva_reorder_pool": ([vp, vp, vp, _Geom, vp], ctypes.c_int),
         "fva_sasa_workspace_size": ([_Geom], sz),
         "fva_route_repair_sasa": ([vp, vp, _Geom, f64, i32, i32, f64, vp, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
-        "fva_route_repair_pooled": ([vp, vp, _Geom, f64, i32, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
+        "fva_route_repair_pooled": ([vp, vp, _Geom, f64, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
         "fva_repair_workspace_size": ([_Geom], sz),
         "fva_repair": ([vp, vp, _Geom, i32, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
         "fva_block_sparse_attn": ([vp, vp, vp, vp, vp, vp, _Geom, f32, vp, vp], ctypes.c_int),
         "fva_block_sparse_attn_natural": ([vp, vp, vp, vp, vp, vp, _Geom, f32, vp, vp], ctypes.c_int),
         "fva_get_device_error": ([vp, ctypes.POINTER(i32)], ctypes.c_int),
+        "fva_debug_set_wait_limit": ([i64], ctypes.c_int),
         "fva_last_error": ([], ctypes.c_char_p),
         "fva_launch_count": ([], i64),
         "fva_version": ([], i32),
@@ -239,9 +240,21 @@ def fva_route_repair(qr, kr, g: Geom, p: float, k: int, counts, idx, head_work, 
                                 workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
+def _workspace(workspace, nbytes: int, like: torch.Tensor) -> torch.Tensor:
+    """The caller's workspace, or a fresh device buffer of nbytes (PyTorch allocates it)."""
+    if workspace is not None:
+        return workspace
+    return torch.empty((max(int(nbytes), 256),), dtype=torch.uint8, device=like.device)
+
+
+def _nbytes(t: Optional[torch.Tensor]) -> int:
+    return 0 if t is None else t.numel() * t.element_size()
+
+
 def fva_route_repair_pooled(qbar, kbar, g: Geom, p: float, k: int, counts, idx, head_work, worklist,
-                            topp_mask=None, topk_idx=None, stream=None):
-    """fva_route_repair from block means already computed (fva_reorder_pool)."""
+                            topp_mask=None, topk_idx=None, workspace=None, stream=None):
+    """fva_route_repair from block means already computed (fva_reorder_pool).  workspace:
+    fva_repair_workspace_size(g) bytes (allocated here when not given)."""
     _need(qbar, torch.float64, (g.B, g.H, g.Nb, g.d), "qbar")
     _need(kbar, torch.float64, (g.B, g.H, g.Nb, g.d), "kbar")
     if topp_mask is not None:
@@ -252,9 +265,10 @@ def fva_route_repair_pooled(qbar, kbar, g: Geom, p: float, k: int, counts, idx, 
     _need(idx, torch.int32, (g.B, g.H, g.Nb, g.Nb), "idx")
     _need(head_work, torch.int64, (g.B, g.H), "head_work")
     _need(worklist, torch.int32, (g.B * g.H * g.Nb,), "worklist")
+    ws = _workspace(workspace, fva_repair_workspace_size(g), counts)
     _check(lib.fva_route_repair_pooled(_ptr(qbar), _ptr(kbar), g.c(), float(p), int(k), _ptr(topp_mask),
                                        _ptr(topk_idx), _ptr(counts), _ptr(idx), _ptr(head_work), _ptr(worklist),
-                                       _stream(stream)))
+                                       _ptr(ws), _nbytes(ws), _stream(stream)))
 
 
 def fva_sasa_workspace_size(g: Geom) -> int:
@@ -288,9 +302,9 @@ def fva_repair(topp_mask, topk_idx, g: Geom, k: int, counts, idx, head_work, wor
     _need(idx, torch.int32, (g.B, g.H, g.Nb, g.Nb), "idx")
     _need(head_work, torch.int64, (g.B, g.H), "head_work")
     _need(worklist, torch.int32, (g.B * g.H * g.Nb,), "worklist")
-    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    ws = _workspace(workspace, fva_repair_workspace_size(g), counts)
     _check(lib.fva_repair(_ptr(topp_mask), _ptr(topk_idx), g.c(), int(k), _ptr(counts), _ptr(idx), _ptr(head_work),
-                          _ptr(worklist), _ptr(workspace), ws_bytes, _stream(stream)))
+                          _ptr(worklist), _ptr(ws), _nbytes(ws), _stream(stream)))
 
 
 def fva_block_sparse_attn(qr, kr, vr, counts, idx, worklist, g: Geom, softmax_scale: float, out_r, stream=None):
@@ -326,6 +340,12 @@ def fva_get_device_error(stream=None) -> int:
     if rc == FVA_ERR_CUDA:
         raise FvaError(rc, lib.fva_last_error().decode())
     return int(code.value)
+
+
+def fva_debug_set_wait_limit(cycles: int) -> None:
+    """Test only: pipeline wait limit (SM cycles) of the attention launches that follow;
+    0 restores the default."""
+    _check(lib.fva_debug_set_wait_limit(int(cycles)))
 
 
 def fva_last_error() -> str:
@@ -381,6 +401,7 @@ class SparseAttention:
                                  torch.empty((g.B, g.H), dtype=torch.int64, device=dev),
                                  torch.empty((g.B * g.H * g.Nb,), dtype=torch.int32, device=dev))
         self.ws = torch.empty((max(fva_route_workspace_size(g), 256),), dtype=torch.uint8, device=dev)
+        self.rws = torch.empty((max(fva_repair_workspace_size(g), 256),), dtype=torch.uint8, device=dev)
         self.qbar, self.kbar = (torch.empty((g.B, g.H, g.Nb, g.d), dtype=torch.float64, device=dev)
                                 for _ in range(2))
 
@@ -388,12 +409,12 @@ class SparseAttention:
         g = self.g
         if self.fused:   # the means come from the reorder pass (reorder_qk)
             fva_route_repair_pooled(self.qbar, self.kbar, g, self.p, self.k, self.rep.counts, self.rep.idx,
-                                    self.rep.head_work, self.rep.worklist, stream=stream)
+                                    self.rep.head_work, self.rep.worklist, workspace=self.rws, stream=stream)
             return
         fva_route(self.qr, self.kr, g, self.p, self.k, self.route.topp_mask, self.route.topk_idx, self.ws,
                   stream=stream)
         fva_repair(self.route.topp_mask, self.route.topk_idx, g, self.k, self.rep.counts, self.rep.idx,
-                   self.rep.head_work, self.rep.worklist, stream=stream)
+                   self.rep.head_work, self.rep.worklist, workspace=self.rws, stream=stream)
 
     def attention(self, stream=None) -> None:
         """Tile-major output into self.outr."""

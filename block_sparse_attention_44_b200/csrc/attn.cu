@@ -16,33 +16,24 @@
 //               quarter, each owning half of the columns of its 32 query rows
 // One thread can issue a tcgen05.mma only about as fast as a 128x128x16 product
 // runs, so the two kinds of product come from two warps on different SM
-// sub-partitions and neither waits for the other's completion: tensor memory holds
-// two S buffers (S_{j+1} is computed while the softmax works on S_j), a separate
-// bf16 P buffer and the fp32 O accumulator.  Online softmax in base 2 with a lazy
-// running max: O and the row sums are rescaled only when the max grows by more
-// than 2^8; a quarter of the exponentials run on the FMA pipe (exp2_poly).
-// Every wait is bounded; on expiry the CTA drains its in-flight copies/MMAs, frees
-// TMEM and reports kDevErrTimeout through the device error word.
+// sub-partitions and neither waits for the other's completion.  Tensor memory holds
+// two S buffers and two bf16 P buffers besides the fp32 O accumulator (all 512
+// columns at d = S = 128): S_{j+2} is issued as soon as the softmax has read S_j out,
+// and the softmax writes P_j while P_{j-1} V_{j-1} may still run, so it never waits
+// for a PV product except to rescale O.  Online softmax in base 2 with a lazy running
+// max: O and the row sums are rescaled only when the max grows by more than 2^8; a
+// quarter of the exponentials run on the FMA pipe (exp2_poly).
+// Every wait is bounded; on expiry the CTA aborts, every role waits for the copies and
+// products it issued, TMEM is freed, and kDevErrTimeout goes to the device error word.
 #include <stdio.h>
+
+#include <atomic>
 
 #include "fva_common.cuh"
 #include "fva_internal.h"
 
 namespace fva {
 namespace {
-
-#ifdef FVA_ATTN_TRACE
-// Profiling build only: clock64() stamps of pipeline events of CTA 0, by block sequence.
-__device__ unsigned long long g_attn_trace[20][4096];
-#define FVA_TRACE(ev, idx)                                         \
-  do {                                                             \
-    if (blockIdx.x == 0 && (idx) < 4096) g_attn_trace[ev][idx] = clock64(); \
-  } while (0)
-#else
-#define FVA_TRACE(ev, idx) \
-  do {                     \
-  } while (0)
-#endif
 
 constexpr int kAttnThreads = 384;   // 12 warps: 4 control + 8 softmax
 constexpr int kBM = 128;               // MMA M: query rows per tile (S=64 tiles use the top half)
@@ -62,13 +53,14 @@ struct AttnCfg {
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
   static constexpr int OFF_V = OFF_K + NSK * KV_BYTES;
   static constexpr int OFF_BAR = OFF_V + NSV * KV_BYTES;
-  // barriers: q_full q_empty s_full[2] s_free[2] p_full[2] o_done o_free drain_s drain_pv; k ring; v ring
-  static constexpr int NBAR = 12 + 2 * NSK + 2 * NSV;
+  // barriers: q_full q_empty s_full[2] s_free[2] p_full[2] o_done[2] o_free drain_s drain_pv; k ring; v ring
+  static constexpr int NBAR = 13 + 2 * NSK + 2 * NSV;
   static constexpr int OFF_RED = OFF_BAR + NBAR * 8;         // row maxima / sums [2 parity][2 half][128]
   static constexpr int OFF_MISC = OFF_RED + 2 * 2 * kBM * 4; // tmem base slot, abort flag
   static constexpr int SMEM = OFF_MISC + 16;                 // base must be 1024-aligned (checked)
-  // TMEM columns: S double buffer [0, 2*BN), P [2*BN, 2*BN + BN/2) as bf16 pairs, O after it
-  static constexpr int T_S = 0, T_P = 2 * BN, T_O = 2 * BN + BN / 2;
+  // TMEM columns: S double buffer [0, 2*BN), P double buffer [2*BN, 3*BN) as bf16 pairs
+  // (BN/2 columns each), O after it
+  static constexpr int T_S = 0, T_P = 2 * BN, T_O = 3 * BN;
   static constexpr int TMEM_USED = T_O + D;
   static constexpr int TMEM_COLS = TMEM_USED <= 128 ? 128 : TMEM_USED <= 256 ? 256 : 512;
   static constexpr uint32_t IDESC_S = idesc_bf16_f32(kBM, BN, false);
@@ -91,6 +83,7 @@ struct AttnParams {
   // reorder fused into the epilogue); grid X, Y and tile tt x ty x tx, nY x nX tiles
   int natural, Y, X, tt, ty, tx, nY, nX;
   const int32_t* order;   // tile numbering table (raster index of tile i), or nullptr
+  long long wait_limit;   // cycles one pipeline wait may take before the CTA aborts
 };
 
 // Token position of row r of tile i in the output: tile-major i*S + r, or the natural
@@ -135,14 +128,6 @@ __device__ __forceinline__ int block_id(const AttnParams& prm, int item, int i, 
   return j;
 }
 
-// Bounded wait that ignores the abort flag (used only while draining).
-__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
-  const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > kWaitLimitCycles / 4) break;
-  }
-}
-
 // One TMA producer warp: one tile (K or V, 64-column boxes) per kept block through an
 // ns-stage ring; the K producer also loads each item's Q.  The whole warp walks the
 // loop and waits (warp-uniform); lane 0 issues.
@@ -162,7 +147,9 @@ __device__ void produce(const AttnParams& prm, const CUtensorMap* tm, const CUte
     const int i = item - static_cast<int>(bh * Nb);
     const long long row0 = bh * prm.N;
     if (WITH_Q) {
-      if (q_items > 0 && !(ok = __all_sync(0xffffffffu, mbar_wait(q_empty, (q_items - 1) & 1, abort_flag)))) break;
+      if (q_items > 0 &&
+          !(ok = __all_sync(0xffffffffu, mbar_wait(q_empty, (q_items - 1) & 1, abort_flag, prm.wait_limit))))
+        break;
       if (leader) {
         mbar_arrive_expect_tx(q_full, Cfg::Q_TX);
         for (int ch = 0; ch < Cfg::NCH; ++ch)
@@ -173,7 +160,8 @@ __device__ void produce(const AttnParams& prm, const CUtensorMap* tm, const CUte
     }
     for (int jj = 0; jj < n; ++jj, ++g) {
       const int st = static_cast<int>(g % NS);
-      if (g >= NS && !(ok = __all_sync(0xffffffffu, mbar_wait(empty0 + 8 * st, ((g / NS) - 1) & 1, abort_flag))))
+      if (g >= NS && !(ok = __all_sync(0xffffffffu, mbar_wait(empty0 + 8 * st, ((g / NS) - 1) & 1, abort_flag,
+                                                              prm.wait_limit))))
         break;
       if (leader) {
         const int j = block_id(prm, item, i, jj, WITH_Q);
@@ -185,9 +173,12 @@ __device__ void produce(const AttnParams& prm, const CUtensorMap* tm, const CUte
       __syncwarp();
     }
   }
-  if (!ok && leader) {
-    // let the copies already issued land before the CTA goes away
-    set_device_error(prm.dev_err, kDevErrTimeout);
+  if (leader) {
+    if (!ok) set_device_error(prm.dev_err, kDevErrTimeout);
+    // every copy issued lands before the CTA goes away, whether this role, another one
+    // or nobody aborted: the last copy into each stage (earlier ones completed before
+    // the stage was refilled) and the last Q.  On a normal exit the consumers already
+    // waited for all of them, so these waits return at once.
     for (long long q = (g > NS ? g - NS : 0); q < g; ++q) drain_wait(full0 + 8 * (q % NS), (q / NS) & 1);
     if (WITH_Q && q_items > 0) drain_wait(q_full, (q_items - 1) & 1);
   }
@@ -211,9 +202,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t sV = sbase + C::OFF_V;
   const uint32_t bar0 = sbase + C::OFF_BAR;
   const uint32_t q_full = bar0, q_empty = bar0 + 8, s_full0 = bar0 + 16, s_free0 = bar0 + 32;
-  const uint32_t p_full0 = bar0 + 48, o_done = bar0 + 64, o_free = bar0 + 72, drain_s = bar0 + 80;
-  const uint32_t drain_pv = bar0 + 88;
-  const uint32_t k_full0 = bar0 + 96;
+  const uint32_t p_full0 = bar0 + 48, o_done0 = bar0 + 64, o_free = bar0 + 80, drain_s = bar0 + 88;
+  const uint32_t drain_pv = bar0 + 96;
+  const uint32_t k_full0 = bar0 + 104;
   const uint32_t k_empty0 = k_full0 + 8 * NSK;
   const uint32_t v_full0 = k_empty0 + 8 * NSK;
   const uint32_t v_empty0 = v_full0 + 8 * NSV;
@@ -230,8 +221,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(s_full0 + 8 * b, 1);
       mbar_init(s_free0 + 8 * b, 256);
       mbar_init(p_full0 + 8 * b, 256);
+      mbar_init(o_done0 + 8 * b, 1);
     }
-    mbar_init(o_done, 1);
     mbar_init(o_free, 256);
     mbar_init(drain_s, 1);
     mbar_init(drain_pv, 1);
@@ -272,8 +263,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int Nb = prm.Nb;
   const int S = BN;
   const bool leader = lane == 0;
+  const long long wlim = prm.wait_limit;
   auto wait_all = [&](uint32_t bar, uint32_t parity) {
-    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, wlim));
   };
 
   if (warp == 0) {
@@ -284,7 +276,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     produce<D, BN, NSV, false, C>(prm, &tmV, &tmQ, sV, v_full0, v_empty0, sQ, q_full, q_empty, abort_flag);
   } else if (warp == 1) {
     // ---------------------------------------------------------------- S issuer
-    // S_j = Q K_j^T into S buffer j % 2 once the softmax has read S_{j-2} out of it.
+    // S_j = Q K_j^T into S buffer j % 2 as soon as the softmax has read S_{j-2} out of it.
     // (One thread issues a tcgen05.mma only every ~50 cycles, about the time a
     // 128x128x16 product takes, so S and PV products come from two warps on
     // different SM sub-partitions.)  The whole warp walks the loop and waits; lane 0
@@ -304,13 +296,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       for (int jj = 0; jj < n; ++jj, ++g) {
         const int b = static_cast<int>(g & 1);
         const int st = static_cast<int>(g % NSK);
-        // S_g is issued when the softmax hands over P_{g-2} (buffer b is free by then, and
-        // P_{g-2} V_{g-2} is issued at the same moment): running S further ahead would
-        // only queue it in front of the PV product the softmax waits on
-        if (g >= 2 && !(ok = wait_all(p_full0 + 8 * b, ((g >> 1) - 1) & 1))) break;
-        if (leader) FVA_TRACE(4, g);
+        // S buffer b is free once the softmax has loaded S_{g-2}; the softmax never waits
+        // on a PV product before writing P (P is double-buffered), so running S up to two
+        // blocks ahead only keeps the tensor pipe fed
+        if (g >= 2 && !(ok = wait_all(s_free0 + 8 * b, ((g >> 1) - 1) & 1))) break;
         if (!(ok = wait_all(k_full0 + 8 * st, (g / NSK) & 1))) break;
-        if (leader) FVA_TRACE(9, g);
         if (leader) {
           tc_fence_after();
           const uint64_t dK = dK0 + static_cast<uint64_t>((st * C::KV_BYTES) >> 4);
@@ -324,7 +314,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           umma_commit(k_empty0 + 8 * st);
           umma_commit(s_full0 + 8 * b);
           if (jj == n - 1) umma_commit(q_empty);   // last reader of this item's Q
-          FVA_TRACE(5, g);
         }
         __syncwarp();
         issued = true;
@@ -338,7 +327,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   } else if (warp == 2) {
     // ---------------------------------------------------------------- PV issuer
-    // O += P_j V_j once the softmax has written P_j (p_full).
+    // O += P_j V_j once the softmax has written P_j into P buffer j % 2 (p_full); the
+    // commit on o_done[j % 2] tells the softmax that buffer and O are free again.
     const uint64_t dV0 = sdesc_sw128(sV, C::KV_CHUNK, 1024);
     long long g = 0, items = 0;
     bool ok = true, issued = false;
@@ -350,20 +340,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       for (int jj = 0; jj < n; ++jj, ++g) {
         const int st = static_cast<int>(g % NSV);
         if (!(ok = wait_all(p_full0 + 8 * static_cast<int>(g & 1), (g >> 1) & 1))) break;
-        if (leader) FVA_TRACE(6, g);
         if (!(ok = wait_all(v_full0 + 8 * st, (g / NSV) & 1))) break;
-        if (leader) FVA_TRACE(10, g);
         if (leader) {
           tc_fence_after();
           const uint64_t dV = dV0 + static_cast<uint64_t>((st * C::KV_BYTES) >> 4);
-          const uint32_t aP = tmem + C::T_P;
+          const uint32_t aP = tmem + C::T_P + static_cast<uint32_t>(g & 1) * (BN / 2);
 #pragma unroll
           for (int ks = 0; ks < BN / 16; ++ks)
             umma_ts(tmem + C::T_O, aP + ks * 8, dV + ((ks * 16 * 128) >> 4), C::IDESC_PV,
                     (jj > 0 || ks > 0) ? 1u : 0u);
           umma_commit(v_empty0 + 8 * st);
-          umma_commit(o_done);
-          FVA_TRACE(7, g);
+          umma_commit(o_done0 + 8 * static_cast<uint32_t>(g & 1));
         }
         __syncwarp();
         issued = true;
@@ -391,19 +378,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int row = quarter * 32 + lane;                          // TMEM lane == query row
     const int pair_bar = 1 + quarter;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t tP = tmem + C::T_P + half * (HB / 2) + lane_off;
+    const uint32_t tP0 = tmem + C::T_P + half * (HB / 2) + lane_off;   // P buffer 0; buffer 1 is BN/2 further
     const uint32_t tO = tmem + C::T_O + half * HD + lane_off;
     float* red_max = reinterpret_cast<float*>(smem + C::OFF_RED);         // [2][2][kBM]
     const float sl2 = prm.scale_log2;
     const uint64_t sl2x2 = f32x2_pack(sl2, sl2);
-    long long g = 0, o_cnt = 0;    // blocks processed; o_done phases observed
+    long long g = 0;   // blocks processed
     bool ok = true;
-    // observe o_done phases up to `upto` (the PV products of blocks <= upto are done)
-    auto need_o = [&](long long upto) {
-      while (ok && o_cnt <= upto) {
-        ok = __all_sync(0xffffffffu, mbar_wait(o_done, o_cnt & 1, abort_flag));
-        ++o_cnt;
-      }
+    // wait until P_q V_q has completed (its commit on o_done[q % 2] is that barrier's
+    // phase q / 2; P_{q+2} V_{q+2} cannot start before this warp writes P_{q+2}, so the
+    // barrier is never two phases ahead of the one waited for)
+    auto wait_pv = [&](long long q) {
+      if (ok && q >= 0)
+        ok = __all_sync(0xffffffffu, mbar_wait(o_done0 + 8 * static_cast<uint32_t>(q & 1), (q >> 1) & 1, abort_flag,
+                                               wlim));
     };
     for (long long it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
       const int item = item_at(prm, it);
@@ -425,8 +413,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       for (int jj = 0; jj < n; ++jj, ++g) {
         const int b = static_cast<int>(g & 1);
         const int par = b;
-        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(s_full0 + 8 * b, (g >> 1) & 1, abort_flag));
-        if (warp == 4 && lane == 0) FVA_TRACE(0, g);
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(s_full0 + 8 * b, (g >> 1) & 1, abort_flag, wlim));
         uint32_t r[HB];
         float pm = -INFINITY;
         if (ok) {
@@ -448,7 +435,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         ok = bar_and(pair_bar, 64, ok);                           // both halves' maxima published
         if (!ok) break;
-        if (warp == 4 && lane == 0) FVA_TRACE(1, g);
         const float m_cand = fmaxf(pm, red_max[(par * 2 + (half ^ 1)) * kBM + row]) * sl2;
         float alpha = 1.0f;
         if (m_cand > m + kLazyRescaleLog2) {
@@ -472,19 +458,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         float a0, a1;
         f32x2_unpack(fadd2(fadd2(rs[0], rs[1]), fadd2(rs[2], rs[3])), a0, a1);
         l = l * alpha + (a0 + a1);
-        if (warp == 4 && lane == 0) FVA_TRACE(2, g);
-        // P and O are read / written by P_{g-1} V_{g-1}: wait for it before touching them
-        need_o(g - 1);
-        if (warp == 4 && lane == 0) FVA_TRACE(8, g);
+        // P buffer b last fed P_{g-2} V_{g-2}; O must hold every earlier product before
+        // it is rescaled (rare: only when the max grows by more than 2^8)
+        const bool rescale = jj > 0 && __any_sync(0xffffffffu, alpha != 1.0f);
+        wait_pv(g - 2);
+        if (rescale) wait_pv(g - 1);
         if (ok) {
           tc_fence_after();
+          const uint32_t tP = tP0 + static_cast<uint32_t>(b) * (BN / 2);
           if constexpr (HB / 2 >= 32) {
 #pragma unroll
             for (int c = 0; c < HB / 64; ++c) tmem_st32(tP + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
           } else {
             tmem_st16(tP, r);
           }
-          if (jj > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+          if (rescale) {
 #pragma unroll
             for (int c = 0; c < HD / 32; ++c) {
               uint32_t o[32];
@@ -498,14 +486,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           tmem_wait_st();
           tc_fence_before();
           mbar_arrive(p_full0 + 8 * b);
-          if (warp == 4 && lane == 0) FVA_TRACE(3, g);
         }
       }
       // no early exit before these barriers: the partner warp must meet them too.  The
       // row sums go through the parity region the next block will use; both warps
       // are past their last reads of it, and the second barrier keeps the next
       // block's maxima from overwriting it before both have read it.
-      need_o(g - 1);
+      wait_pv(g - 1);                                             // the item's last product is in O
       float* red_l = red_max + (g & 1) * 2 * kBM;
       red_l[half * kBM + row] = l;
       ok = bar_and(pair_bar, 64, ok);
@@ -579,6 +566,9 @@ bool make_map(CUtensorMap* m, const void* base, long long rows, int D, int box_r
   return true;
 }
 
+// Pipeline wait limit of the next launches (0: kWaitLimitCycles); only a test changes it.
+std::atomic<long long> g_wait_limit{0};
+
 int sm_count() {
   static int n = 0;
   if (!n) {
@@ -605,6 +595,8 @@ cudaError_t launch_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
 }
 
 }  // namespace
+
+void set_attn_wait_limit(long long cycles) { g_wait_limit.store(cycles > 0 ? cycles : 0); }
 
 cudaError_t launch_attention(const void* qr, const void* kr, const void* vr, const int32_t* counts, const int32_t* idx,
                              const int32_t* worklist, const Dims& D, const fva_geom* natural, float scale, void* out,
@@ -633,6 +625,8 @@ cudaError_t launch_attention(const void* qr, const void* kr, const void* vr, con
   prm.nY = D.nY;
   prm.nX = D.nX;
   prm.order = natural ? D.order : nullptr;
+  const long long wl = g_wait_limit.load();
+  prm.wait_limit = wl > 0 ? wl : kWaitLimitCycles;
   cudaError_t e;
   if (D.d == 128 && D.S == 128)
     e = launch_t<128, 128, 3, 3>(mq, mk, mv, prm, s);
@@ -648,8 +642,3 @@ cudaError_t launch_attention(const void* qr, const void* kr, const void* vr, con
 
 }  // namespace fva
 
-#ifdef FVA_ATTN_TRACE
-extern "C" int fva_debug_attn_trace(unsigned long long* host_out) {
-  return cudaMemcpyFromSymbol(host_out, fva::g_attn_trace, sizeof(fva::g_attn_trace)) == cudaSuccess ? 0 : 3;
-}
-#endif

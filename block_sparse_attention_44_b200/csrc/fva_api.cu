@@ -6,6 +6,7 @@
 
 #include <algorithm>
 #include <atomic>
+#include <mutex>
 #include <utility>
 #include <vector>
 
@@ -17,7 +18,12 @@ namespace {
 thread_local char g_err[512] = "";
 std::atomic<long long> g_launches{0};
 
-__device__ int g_dev_err = 0;   // device error word (fva::kDevErr*)
+// Device error words (fva::kDevErr*), one per stream: the first kErrSlots - 1 distinct
+// streams a process launches on (per device) each get a word of their own; any further
+// stream shares word 0.  A kernel reports into the word of the stream it runs on, and
+// fva_get_device_error(stream) reads and clears that word only.
+constexpr int kErrSlots = 64;
+__device__ int g_dev_err[kErrSlots];
 
 int fail(int code, const char* fmt, ...) {
   va_list ap;
@@ -31,17 +37,26 @@ int cuda_fail(cudaError_t e, const char* where) {
   return fail(FVA_ERR_CUDA, "%s: %s (%s)", where, cudaGetErrorName(e), cudaGetErrorString(e));
 }
 
-int* dev_err_ptr() {
-  // per device: the symbol's address differs between devices
-  static int* ptrs[64] = {nullptr};
+// Error word of `stream` on the current device (nullptr if the runtime cannot say).
+int* dev_err_ptr(void* stream) {
+  constexpr int kMaxDev = 64;
+  static std::mutex mu;
+  static int* base[kMaxDev] = {nullptr};                 // the array's address differs per device
+  static std::vector<std::pair<void*, int>> slots[kMaxDev];
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  if (!ptrs[dev]) {
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!base[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_dev_err) != cudaSuccess) return nullptr;
-    ptrs[dev] = static_cast<int*>(p);
+    base[dev] = static_cast<int*>(p);
   }
-  return ptrs[dev];
+  for (const auto& e : slots[dev])
+    if (e.first == stream) return base[dev] + e.second;
+  const int slot = static_cast<int>(slots[dev].size()) + 1;
+  if (slot >= kErrSlots) return base[dev];                // table full: the shared word
+  slots[dev].emplace_back(stream, slot);
+  return base[dev] + slot;
 }
 
 // Validates the geometry; fills D.  Returns FVA_OK or an error code (message set).
@@ -120,7 +135,7 @@ int finish(cudaError_t e, int launches, const char* where) {
 
 extern "C" {
 
-int32_t fva_version(void) { return 105; }
+int32_t fva_version(void) { return 200; }
 
 const char* fva_last_error(void) { return g_err; }
 
@@ -166,7 +181,7 @@ static int reorder_common(const void* src, void* dst, fva_geom g, void* stream, 
   if (!src || !dst) return fail(FVA_ERR_INVALID_ARG, "null tensor pointer");
   if (src == dst) return fail(FVA_ERR_INVALID_ARG, "in-place reorder is not supported");
   if (!aligned16(src) || !aligned16(dst)) return fail(FVA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
-  int* de = dev_err_ptr();
+  int* de = dev_err_ptr(stream);
   if (!de) return fail(FVA_ERR_CUDA, "reorder: cannot resolve the device error word");
   int launches = 0;
   cudaError_t e = fva::launch_reorder(src, dst, g, D, inverse, de, static_cast<cudaStream_t>(stream), &launches);
@@ -187,17 +202,29 @@ int fva_reorder_pool(const void* x, void* xr, double* pooled, fva_geom g, void* 
   if (x == xr) return fail(FVA_ERR_INVALID_ARG, "in-place reorder is not supported");
   if (!aligned16(x) || !aligned16(xr)) return fail(FVA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
   if ((reinterpret_cast<uintptr_t>(pooled) & 7u) != 0) return fail(FVA_ERR_INVALID_ARG, "pooled must be 8-byte aligned");
-  int* de = dev_err_ptr();
+  int* de = dev_err_ptr(stream);
   if (!de) return fail(FVA_ERR_CUDA, "fva_reorder_pool: cannot resolve the device error word");
   int launches = 0;
   cudaError_t e = fva::launch_reorder_pool(x, xr, pooled, g, D, de, static_cast<cudaStream_t>(stream), &launches);
   return finish(e, launches, "fva_reorder_pool");
 }
 
+// Workspace of the routing calls: the float64 block means, then the LPT scratch.
+static size_t route_ws_total(const fva::Dims& D) { return fva::route_workspace_bytes(D) + fva::lpt_workspace_bytes(D); }
+
 size_t fva_route_workspace_size(fva_geom g) {
   fva::Dims D;
   if (check_geom(g, D, false)) return 0;
-  return fva::route_workspace_bytes(D);
+  return route_ws_total(D);
+}
+
+// Checks a caller workspace of at least `need` bytes; FVA_OK or an error (message set).
+static int check_ws(const void* ws, size_t ws_bytes, size_t need) {
+  if (!ws) return fail(FVA_ERR_INVALID_ARG, "null workspace");
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return fail(FVA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (ws_bytes < need)
+    return fail(FVA_ERR_INVALID_ARG, "workspace too small: %zu bytes given, %zu needed", ws_bytes, need);
+  return FVA_OK;
 }
 
 int fva_route(const void* qr, const void* kr, fva_geom g, double p, int32_t k, uint8_t* topp_mask, int32_t* topk_idx,
@@ -205,16 +232,12 @@ int fva_route(const void* qr, const void* kr, fva_geom g, double p, int32_t k, u
   fva::Dims D;
   int rc = check_geom(g, D, false);
   if (rc) return rc;
-  if (!qr || !kr || !topp_mask || !topk_idx || !workspace) return fail(FVA_ERR_INVALID_ARG, "null pointer");
+  if (!qr || !kr || !topp_mask || !topk_idx) return fail(FVA_ERR_INVALID_ARG, "null pointer");
   if (!(p > 0.0) || !(p <= 1.0)) return fail(FVA_ERR_INVALID_ARG, "p must satisfy 0 < p <= 1 (got %g)", p);
   if (k < 1) return fail(FVA_ERR_INVALID_ARG, "k must be >= 1 (got %d)", k);
   if (D.Nb > fva::kMaxNb) return fail(FVA_ERR_UNSUPPORTED, "Nb = %d blocks exceeds %d", D.Nb, fva::kMaxNb);
   if (!aligned16(qr) || !aligned16(kr)) return fail(FVA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
-  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
-    return fail(FVA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
-  const size_t need = fva::route_workspace_bytes(D);
-  if (workspace_bytes < need)
-    return fail(FVA_ERR_INVALID_ARG, "workspace too small: %zu bytes given, %zu needed", workspace_bytes, need);
+  if ((rc = check_ws(workspace, workspace_bytes, route_ws_total(D)))) return rc;
   const int kk = k < D.Nb ? k : D.Nb;
   int launches = 0;
   cudaError_t e = fva::launch_route(qr, kr, D, p, kk, topp_mask, topk_idx, logits_out, nullptr, nullptr, workspace,
@@ -228,29 +251,26 @@ int fva_route_repair(const void* qr, const void* kr, fva_geom g, double p, int32
   fva::Dims D;
   int rc = check_geom(g, D, false);
   if (rc) return rc;
-  if (!qr || !kr || !counts || !idx || !head_work || !worklist || !workspace)
-    return fail(FVA_ERR_INVALID_ARG, "null pointer");
+  if (!qr || !kr || !counts || !idx || !head_work || !worklist) return fail(FVA_ERR_INVALID_ARG, "null pointer");
   if (!(p > 0.0) || !(p <= 1.0)) return fail(FVA_ERR_INVALID_ARG, "p must satisfy 0 < p <= 1 (got %g)", p);
   if (k < 1) return fail(FVA_ERR_INVALID_ARG, "k must be >= 1 (got %d)", k);
   if (D.Nb > fva::kMaxNb) return fail(FVA_ERR_UNSUPPORTED, "Nb = %d blocks exceeds %d", D.Nb, fva::kMaxNb);
   if (!aligned16(qr) || !aligned16(kr)) return fail(FVA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
-  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
-    return fail(FVA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
-  const size_t need = fva::route_workspace_bytes(D);
-  if (workspace_bytes < need)
-    return fail(FVA_ERR_INVALID_ARG, "workspace too small: %zu bytes given, %zu needed", workspace_bytes, need);
+  if ((rc = check_ws(workspace, workspace_bytes, route_ws_total(D)))) return rc;
   const int kk = k < D.Nb ? k : D.Nb;
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  void* lpt_ws = static_cast<unsigned char*>(workspace) + fva::route_workspace_bytes(D);
   int launches = 0;
   cudaError_t e = fva::launch_route(qr, kr, D, p, kk, topp_mask, topk_idx, nullptr, counts, idx, workspace, s,
                                     &launches);
-  if (e == cudaSuccess) e = fva::launch_lpt(counts, D, head_work, worklist, s, &launches);
+  if (e == cudaSuccess) e = fva::launch_lpt(counts, D, head_work, worklist, lpt_ws, s, &launches);
   return finish(e, launches, "fva_route_repair");
 }
 
 int fva_route_repair_pooled(const double* qbar, const double* kbar, fva_geom g, double p, int32_t k,
                             uint8_t* topp_mask, int32_t* topk_idx, int32_t* counts, int32_t* idx,
-                            int64_t* head_work, int32_t* worklist, void* stream) {
+                            int64_t* head_work, int32_t* worklist, void* workspace, size_t workspace_bytes,
+                            void* stream) {
   fva::Dims D;
   int rc = check_geom(g, D, false);
   if (rc) return rc;
@@ -259,19 +279,22 @@ int fva_route_repair_pooled(const double* qbar, const double* kbar, fva_geom g, 
   if (k < 1) return fail(FVA_ERR_INVALID_ARG, "k must be >= 1 (got %d)", k);
   if (D.Nb > fva::kMaxNb) return fail(FVA_ERR_UNSUPPORTED, "Nb = %d blocks exceeds %d", D.Nb, fva::kMaxNb);
   if (!aligned16(qbar) || !aligned16(kbar)) return fail(FVA_ERR_INVALID_ARG, "qbar and kbar must be 16-byte aligned");
+  if ((rc = check_ws(workspace, workspace_bytes, fva::lpt_workspace_bytes(D)))) return rc;
   const int kk = k < D.Nb ? k : D.Nb;
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   int launches = 0;
   cudaError_t e = fva::launch_select_pooled(qbar, kbar, D, p, kk, topp_mask, topk_idx, nullptr, counts, idx, s,
                                             &launches);
-  if (e == cudaSuccess) e = fva::launch_lpt(counts, D, head_work, worklist, s, &launches);
+  if (e == cudaSuccess) e = fva::launch_lpt(counts, D, head_work, worklist, workspace, s, &launches);
   return finish(e, launches, "fva_route_repair_pooled");
 }
+
+static size_t sasa_lpt_offset(const fva::Dims& D) { return (fva::sasa_workspace_bytes(D) + 255) & ~static_cast<size_t>(255); }
 
 size_t fva_sasa_workspace_size(fva_geom g) {
   fva::Dims D;
   if (check_geom(g, D, false)) return 0;
-  return fva::sasa_workspace_bytes(D);
+  return sasa_lpt_offset(D) + fva::lpt_workspace_bytes(D);
 }
 
 int fva_route_repair_sasa(const double* qbar, const double* kbar, fva_geom g, double p, int32_t k, int32_t num_ranks,
@@ -290,29 +313,26 @@ int fva_route_repair_sasa(const double* qbar, const double* kbar, fva_geom g, do
   if (!(alpha >= 0.0) || !(alpha <= 1.0)) return fail(FVA_ERR_INVALID_ARG, "alpha must lie in [0, 1] (got %g)", alpha);
   if (D.Nb > fva::kMaxNb) return fail(FVA_ERR_UNSUPPORTED, "Nb = %d blocks exceeds %d", D.Nb, fva::kMaxNb);
   if (!aligned16(qbar) || !aligned16(kbar)) return fail(FVA_ERR_INVALID_ARG, "qbar and kbar must be 16-byte aligned");
-  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
-    return fail(FVA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
-  const size_t need = fva::sasa_workspace_bytes(D);
-  if (workspace_bytes < need)
-    return fail(FVA_ERR_INVALID_ARG, "workspace too small: %zu bytes given, %zu needed", workspace_bytes, need);
+  if ((rc = check_ws(workspace, workspace_bytes, sasa_lpt_offset(D) + fva::lpt_workspace_bytes(D)))) return rc;
   const int kk = k < D.Nb ? k : D.Nb;
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   int launches = 0;
   cudaError_t e = fva::launch_sasa(qbar, kbar, D, p, kk, num_ranks, alpha, counts, idx, extra, workspace, s,
                                    &launches);
-  if (e == cudaSuccess) e = fva::launch_lpt(counts, D, head_work, worklist, s, &launches);
+  if (e == cudaSuccess)
+    e = fva::launch_lpt(counts, D, head_work, worklist, static_cast<unsigned char*>(workspace) + sasa_lpt_offset(D), s,
+                        &launches);
   return finish(e, launches, "fva_route_repair_sasa");
 }
 
 size_t fva_repair_workspace_size(fva_geom g) {
-  (void)g;
-  return 0;
+  fva::Dims D;
+  if (check_geom(g, D, false)) return 0;
+  return fva::lpt_workspace_bytes(D);
 }
 
 int fva_repair(const uint8_t* topp_mask, const int32_t* topk_idx, fva_geom g, int32_t k, int32_t* counts, int32_t* idx,
                int64_t* head_work, int32_t* worklist, void* workspace, size_t workspace_bytes, void* stream) {
-  (void)workspace;
-  (void)workspace_bytes;
   fva::Dims D;
   int rc = check_geom(g, D, false);
   if (rc) return rc;
@@ -320,11 +340,12 @@ int fva_repair(const uint8_t* topp_mask, const int32_t* topk_idx, fva_geom g, in
     return fail(FVA_ERR_INVALID_ARG, "null pointer");
   if (k < 1) return fail(FVA_ERR_INVALID_ARG, "k must be >= 1 (got %d)", k);
   if (D.Nb > fva::kMaxNb) return fail(FVA_ERR_UNSUPPORTED, "Nb = %d blocks exceeds %d", D.Nb, fva::kMaxNb);
-  int* de = dev_err_ptr();
+  if ((rc = check_ws(workspace, workspace_bytes, fva::lpt_workspace_bytes(D)))) return rc;
+  int* de = dev_err_ptr(stream);
   if (!de) return fail(FVA_ERR_CUDA, "fva_repair: cannot resolve the device error word");
   const int kk = k < D.Nb ? k : D.Nb;
   int launches = 0;
-  cudaError_t e = fva::launch_repair(topp_mask, topk_idx, D, kk, counts, idx, head_work, worklist, de,
+  cudaError_t e = fva::launch_repair(topp_mask, topk_idx, D, kk, counts, idx, head_work, worklist, workspace, de,
                                      static_cast<cudaStream_t>(stream), &launches);
   return finish(e, launches, "fva_repair");
 }
@@ -340,7 +361,7 @@ static int attn_common(const void* qr, const void* kr, const void* vr, const int
     return fail(FVA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
   if (!isfinite(softmax_scale)) return fail(FVA_ERR_INVALID_ARG, "softmax_scale must be finite");
   const float scale = softmax_scale > 0.0f ? softmax_scale : 1.0f / sqrtf(static_cast<float>(D.d));
-  int* de = dev_err_ptr();
+  int* de = dev_err_ptr(stream);
   if (!de) return fail(FVA_ERR_CUDA, "%s: cannot resolve the device error word", name);
   char msg[256] = "";
   int launches = 0;
@@ -366,10 +387,16 @@ int fva_block_sparse_attn_natural(const void* qr, const void* kr, const void* vr
                      "fva_block_sparse_attn_natural");
 }
 
+int fva_debug_set_wait_limit(int64_t cycles) {
+  fva::set_attn_wait_limit(cycles);
+  g_err[0] = '\0';
+  return FVA_OK;
+}
+
 int fva_get_device_error(void* stream, int32_t* code) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "fva_get_device_error");
-  int* de = dev_err_ptr();
+  int* de = dev_err_ptr(stream);
   if (!de) return fail(FVA_ERR_CUDA, "fva_get_device_error: cannot resolve the device error word");
   int v = 0;
   e = cudaMemcpy(&v, de, sizeof(int), cudaMemcpyDeviceToHost);
@@ -431,7 +458,7 @@ extern "C" int fva_route_static(const void* qr, const void* kr, fva_geom g, doub
   if (k < 1) return fail(FVA_ERR_INVALID_ARG, "k must be >= 1 (got %d)", k);
   if (D.Nb > fva::kMaxNb) return fail(FVA_ERR_UNSUPPORTED, "Nb = %d blocks exceeds %d", D.Nb, fva::kMaxNb);
   if (!aligned16(qr) || !aligned16(kr)) return fail(FVA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
-  const size_t need = fva::route_workspace_bytes(D);
+  const size_t need = route_ws_total(D);   // the size fva_route_workspace_size() reports
   if (need > kRouteStaticScratchBytes)
     return fail(FVA_ERR_UNSUPPORTED,
                 "fva_route_static: this geometry needs %zu bytes of routing scratch, more than the %zu-byte "

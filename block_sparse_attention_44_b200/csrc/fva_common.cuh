@@ -16,8 +16,11 @@ enum : int {
   kDevErrMisaligned = 3,   // dynamic shared memory was not 1024-byte aligned
 };
 
-// Roughly 2 s at 1.9 GHz: no single pipeline wait in these kernels is anywhere near it.
+// Default limit of one pipeline wait: roughly 2 s at 1.9 GHz, far above any wait of a
+// working pipeline.  Waits for copies and products already in flight (drains) always
+// use kDrainLimitCycles, whatever limit the pipeline waits were given.
 constexpr long long kWaitLimitCycles = 4000000000LL;
+constexpr long long kDrainLimitCycles = kWaitLimitCycles / 4;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -47,18 +50,46 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// try_wait that suspends the thread for at most `ns` nanoseconds (instead of the
+// system-dependent time limit of the plain form).
+__device__ __forceinline__ bool mbar_try_wait_ns(uint32_t bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+// Limits below this many cycles are test limits: their waits suspend the thread only
+// briefly, so the limit is checked at that resolution.
+constexpr long long kShortWaitLimit = 1000000;
+
 // Waits for phase `parity` of the barrier.  Gives up (returns false) when *abort is
-// raised by another role or after kWaitLimitCycles, raising *abort itself then.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
-  if (mbar_try_wait(bar, parity)) return true;
+// raised by another role or after `limit` cycles, raising *abort itself then.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
+                                          long long limit = kWaitLimitCycles) {
+  const bool short_limit = limit < kShortWaitLimit;
+  const uint32_t ns = static_cast<uint32_t>(short_limit ? (limit / 4 > 0 ? limit / 4 : 1) : 0);
+  if (short_limit ? mbar_try_wait_ns(bar, parity, ns) : mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (short_limit ? mbar_try_wait_ns(bar, parity, ns) : mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (clock64() - t0 > kWaitLimitCycles) {
+    if (clock64() - t0 > limit) {
       *abort = 1;
       return false;
     }
+  }
+}
+// Bounded wait that ignores the abort flag: only for copies and products already issued
+// (drains), which complete on their own.
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > kDrainLimitCycles) break;
   }
 }
 

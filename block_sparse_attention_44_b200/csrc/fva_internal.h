@@ -39,10 +39,10 @@ cudaError_t launch_select_pooled(const double* qbar, const double* kbar, const D
                                  uint8_t* topp_mask, int32_t* topk_idx, double* logits_out, int32_t* counts,
                                  int32_t* idx, cudaStream_t s, int* launches);
 
-// Repair + compaction + per-head work + LPT work list.
+// Repair + compaction + per-head work + LPT work list (ws: lpt_workspace_bytes).
 cudaError_t launch_repair(const uint8_t* topp_mask, const int32_t* topk_idx, const Dims& D, int kk, int32_t* counts,
-                          int32_t* idx, int64_t* head_work, int32_t* worklist, int* dev_err, cudaStream_t s,
-                          int* launches);
+                          int32_t* idx, int64_t* head_work, int32_t* worklist, void* ws, int* dev_err,
+                          cudaStream_t s, int* launches);
 
 // Slack-aware augmentation from block means: selection (recording each row's ranked
 // prefix), per-row floors from the virtual-rank budgets, selection again with them.
@@ -52,9 +52,15 @@ cudaError_t launch_sasa(const double* qbar, const double* kbar, const Dims& D, d
 size_t sasa_workspace_bytes(const Dims& D);
 constexpr int kMaxVirtualRanks = 1024;
 
-// Per-head work W_h and the LPT work list from the per-row counts.
-cudaError_t launch_lpt(const int32_t* counts, const Dims& D, int64_t* head_work, int32_t* worklist, cudaStream_t s,
-                       int* launches);
+// Per-head work W_h and the LPT work list from the per-row counts; ws holds
+// lpt_workspace_bytes(D) (per-head histograms, then list offsets), 256-byte aligned.
+cudaError_t launch_lpt(const int32_t* counts, const Dims& D, int64_t* head_work, int32_t* worklist, void* ws,
+                       cudaStream_t s, int* launches);
+size_t lpt_workspace_bytes(const Dims& D);
+
+// Pipeline wait limit (cycles) of the attention launches that follow; <= 0 restores
+// the default.  Test-only: lets a test make a wait expire on purpose.
+void set_attn_wait_limit(long long cycles);
 
 // Block-sparse attention (tcgen05).
 // natural != nullptr: O is written in natural token order of that geometry.

@@ -7,8 +7,9 @@
 //
 //   compact_kernel — one warp per (b, h, i) row: kept = Top-p mask | Top-k floor |
 //                    diagonal, written as an ascending id list with ballot/popc.
-//   lpt_kernel     — one CTA per count value (stable counting sort by count,
-//                    descending, without atomics) plus one CTA per head for W_h.
+//   lpt_*_kernel   — W_h and the work list: a stable counting sort of the items by
+//                    count, descending, in three passes (histograms per head, list
+//                    offsets, scatter), without output atomics.
 #include "fva_common.cuh"
 #include "fva_internal.h"
 
@@ -55,91 +56,149 @@ __global__ void __launch_bounds__(kCompactWarps * 32) compact_kernel(const uint8
 }
 
 constexpr int kLptThreads = 256;
+constexpr int kLptScanThreads = 1024;
 
-// Block-wide exclusive prefix sum of v (every thread of a kLptThreads CTA calls it);
-// returns the exclusive prefix and the total in *total.
-__device__ __forceinline__ unsigned block_exclusive_scan(unsigned v, unsigned* total, unsigned* sh) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  unsigned incl = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
-  }
-  if (lane == 31) sh[warp] = incl;
+// Sort key of a count: clamped into [0, Nb] (the attention kernel reads counts the same way).
+__device__ __forceinline__ int lpt_key(int c, int Nb) { return c < 0 ? 0 : (c > Nb ? Nb : c); }
+
+// The LPT work list is a stable counting sort of the items u = bh * Nb + i by count,
+// descending, in three passes over the B*H heads ("chunks" of Nb items), none with
+// output atomics, so the list is deterministic:
+//   lpt_hist_kernel    — per chunk: histogram of its counts over [0, Nb], and W_h;
+//   lpt_offsets_kernel — one CTA: for every count value v (descending) and chunk c
+//                        (ascending), the list position of the first item of chunk c
+//                        with count v, written over the histogram;
+//   lpt_scatter_kernel — per chunk: one warp walks the chunk's items in order, 32 at a
+//                        time; items with equal counts take consecutive positions
+//                        (warp match + running per-value cursors in shared memory).
+// Work is O(B*H*Nb) plus O(B*H*Nb) for the offsets (histogram entries).
+
+// grid.x = BH; hist: [BH][Nb + 1] int32 output; head_work[bh] = sum of the counts.
+__global__ void __launch_bounds__(kLptThreads) lpt_hist_kernel(const int32_t* __restrict__ counts, int Nb,
+                                                               int32_t* __restrict__ hist,
+                                                               int64_t* __restrict__ head_work) {
+  extern __shared__ int h_smem[];
+  __shared__ long long part[kLptThreads / 32];
+  const long long bh = blockIdx.x;
+  for (int v = threadIdx.x; v <= Nb; v += kLptThreads) h_smem[v] = 0;
   __syncthreads();
-  unsigned before = 0, all = 0;
-#pragma unroll
-  for (int w = 0; w < kLptThreads / 32; ++w) {
-    const unsigned t = sh[w];
-    if (w < warp) before += t;
-    all += t;
+  long long s = 0;
+  for (int i = threadIdx.x; i < Nb; i += kLptThreads) {
+    const int c = __ldg(counts + bh * Nb + i);
+    s += c;
+    atomicAdd(&h_smem[lpt_key(c, Nb)], 1);   // order-free counts: deterministic
   }
-  __syncthreads();   // sh may be reused by the caller
-  *total = all;
-  return before + incl - v;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    long long t = 0;
+    for (int w = 0; w < kLptThreads / 32; ++w) t += part[w];
+    head_work[bh] = t;
+  }
+  for (int v = threadIdx.x; v <= Nb; v += kLptThreads) hist[bh * (Nb + 1) + v] = h_smem[v];
 }
 
-// grid.x = (Nb + 1) + BH.  CTA c <= Nb places the items whose count is c: they start
-// after every item with a larger count (descending order) and keep their item order
-// (ties by item id ascending).  Each thread owns a contiguous run of items, counts the
-// larger and equal ones in a first pass over the counts, and after a block scan writes
-// its equal items in order in a second pass.  The remaining BH CTAs write
-// W_h = sum of the counts of head h.  No atomics: the result is deterministic.
-__global__ void __launch_bounds__(kLptThreads) lpt_kernel(const int32_t* __restrict__ counts, long long BH, int Nb,
-                                                          int64_t* __restrict__ head_work,
-                                                          int32_t* __restrict__ worklist) {
-  __shared__ unsigned sh[kLptThreads / 32];
-  __shared__ long long shs[kLptThreads / 32];
-  const long long n = BH * Nb;
-  const int c = static_cast<int>(blockIdx.x);
-  if (c > Nb) {   // realised per-head workload
-    const long long bh = c - (Nb + 1);
-    long long s = 0;
-    for (int i = threadIdx.x; i < Nb; i += kLptThreads) s += __ldg(counts + bh * Nb + i);
+// One CTA.  Thread-owned values v: total[v] = sum over chunks; base[v] = number of items
+// with a larger count (block scan over v descending); then hist[c][v] is replaced by
+// base[v] + sum of hist[c'][v] over chunks c' < c.
+__global__ void __launch_bounds__(kLptScanThreads) lpt_offsets_kernel(int32_t* __restrict__ hist, long long BH,
+                                                                      int Nb) {
+  constexpr int VPT = (kMaxNb + 1 + kLptScanThreads - 1) / kLptScanThreads;   // values per thread
+  __shared__ long long warp_tot[kLptScanThreads / 32];
+  const int V = Nb + 1;
+  // thread t owns the values v = V - 1 - (t * VPT + e), e < VPT: descending order runs
+  // with the thread index, so an exclusive scan over threads gives "larger counts first"
+  long long tot[VPT];
+  long long mine = 0;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if ((threadIdx.x & 31) == 0) shs[threadIdx.x >> 5] = s;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      long long t = 0;
-      for (int w = 0; w < kLptThreads / 32; ++w) t += shs[w];
-      head_work[bh] = t;
+  for (int e = 0; e < VPT; ++e) {
+    const int r = threadIdx.x * VPT + e;   // rank of the value in descending order
+    tot[e] = 0;
+    if (r < V) {
+      const int v = V - 1 - r;
+      for (long long c = 0; c < BH; ++c) tot[e] += hist[c * V + v];
     }
-    return;
+    mine += tot[e];
   }
-  const long long per = (n + kLptThreads - 1) / kLptThreads;
-  const long long lo = threadIdx.x * per;
-  const long long hi = min(n, lo + per);
-  unsigned gt = 0, eq = 0;
-#pragma unroll 8
-  for (long long u = lo; u < hi; ++u) {
-    const int v = __ldg(counts + u);
-    gt += v > c ? 1u : 0u;
-    eq += v == c ? 1u : 0u;
+  // exclusive scan of `mine` over the threads
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  long long incl = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const long long y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
   }
-  unsigned larger, equal;
-  (void)block_exclusive_scan(gt, &larger, sh);
-  unsigned pos = block_exclusive_scan(eq, &equal, sh) + larger;
-  if (equal == 0 || eq == 0) return;   // nothing of this count in this thread's run
-#pragma unroll 8
-  for (long long u = lo; u < hi; ++u)
-    if (__ldg(counts + u) == c) worklist[pos++] = static_cast<int32_t>(u);
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  long long before = 0;
+  for (int w = 0; w < warp; ++w) before += warp_tot[w];
+  long long base = before + incl - mine;
+#pragma unroll
+  for (int e = 0; e < VPT; ++e) {
+    const int r = threadIdx.x * VPT + e;
+    if (r < V) {
+      const int v = V - 1 - r;
+      long long run = base;
+      for (long long c = 0; c < BH; ++c) {
+        const int n = hist[c * V + v];
+        hist[c * V + v] = static_cast<int32_t>(run);
+        run += n;
+      }
+    }
+    base += tot[e];
+  }
+}
+
+// grid.x = BH, one warp per CTA.  off: [BH][Nb + 1] first positions from lpt_offsets_kernel.
+__global__ void __launch_bounds__(32) lpt_scatter_kernel(const int32_t* __restrict__ counts, int Nb,
+                                                         const int32_t* __restrict__ off,
+                                                         int32_t* __restrict__ worklist) {
+  extern __shared__ int cursor[];
+  const long long bh = blockIdx.x;
+  const int lane = threadIdx.x;
+  for (int v = lane; v <= Nb; v += 32) cursor[v] = off[bh * (Nb + 1) + v];
+  __syncwarp();
+  const unsigned lt = (1u << lane) - 1u;
+  for (int i0 = 0; i0 < Nb; i0 += 32) {
+    const int i = i0 + lane;
+    const bool valid = i < Nb;
+    const int key = valid ? lpt_key(__ldg(counts + bh * Nb + i), Nb) : -1 - lane;   // invalid lanes match no one
+    const unsigned peers = __match_any_sync(0xffffffffu, key);
+    if (valid) worklist[cursor[key] + __popc(peers & lt)] = static_cast<int32_t>(bh * Nb + i);
+    __syncwarp();
+    if (valid && (peers & lt) == 0) cursor[key] += __popc(peers);   // the group's first lane advances
+    __syncwarp();
+  }
 }
 
 }  // namespace
 
-cudaError_t launch_lpt(const int32_t* counts, const Dims& D, int64_t* head_work, int32_t* worklist, cudaStream_t s,
-                       int* launches) {
-  const unsigned grid = static_cast<unsigned>(D.Nb + 1 + D.BH());
-  lpt_kernel<<<grid, kLptThreads, 0, s>>>(counts, D.BH(), D.Nb, head_work, worklist);
+size_t lpt_workspace_bytes(const Dims& D) {
+  return (static_cast<size_t>(D.BH()) * (D.Nb + 1) * sizeof(int32_t) + 255) & ~static_cast<size_t>(255);
+}
+
+cudaError_t launch_lpt(const int32_t* counts, const Dims& D, int64_t* head_work, int32_t* worklist, void* ws,
+                       cudaStream_t s, int* launches) {
+  int32_t* hist = static_cast<int32_t*>(ws);
+  const unsigned grid = static_cast<unsigned>(D.BH());
+  const size_t hsmem = static_cast<size_t>(D.Nb + 1) * sizeof(int);
+  lpt_hist_kernel<<<grid, kLptThreads, hsmem, s>>>(counts, D.Nb, hist, head_work);
+  ++*launches;
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  lpt_offsets_kernel<<<1, kLptScanThreads, 0, s>>>(hist, D.BH(), D.Nb);
+  ++*launches;
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  lpt_scatter_kernel<<<grid, 32, hsmem, s>>>(counts, D.Nb, hist, worklist);
   ++*launches;
   return cudaGetLastError();
 }
 
 cudaError_t launch_repair(const uint8_t* topp_mask, const int32_t* topk_idx, const Dims& D, int kk, int32_t* counts,
-                          int32_t* idx, int64_t* head_work, int32_t* worklist, int* dev_err, cudaStream_t s,
-                          int* launches) {
+                          int32_t* idx, int64_t* head_work, int32_t* worklist, void* ws, int* dev_err,
+                          cudaStream_t s, int* launches) {
   const unsigned cgrid = static_cast<unsigned>((D.rows() + kCompactWarps - 1) / kCompactWarps);
   const size_t csmem = static_cast<size_t>(kCompactWarps) * D.Nb;
   compact_kernel<<<cgrid, kCompactWarps * 32, csmem, s>>>(topp_mask, topk_idx, D.rows(), D.Nb, kk, counts, idx,
@@ -147,7 +206,7 @@ cudaError_t launch_repair(const uint8_t* topp_mask, const int32_t* topk_idx, con
   ++*launches;
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  return launch_lpt(counts, D, head_work, worklist, s, launches);
+  return launch_lpt(counts, D, head_work, worklist, ws, s, launches);
 }
 
 }  // namespace fva

@@ -105,7 +105,8 @@ int fva_inverse_reorder(const void* xr, void* x, fva_geom g, void* stream);
  */
 int fva_reorder_pool(const void* x, void* xr, double* pooled, fva_geom g, void* stream);
 
-/* Workspace bytes fva_route needs for geometry g (pooled Q and K, float64). */
+/* Workspace bytes fva_route and fva_route_repair need for geometry g: the float64
+ * pooled Q and K, then the scratch of the LPT work-list sort (as fva_repair's). */
 size_t fva_route_workspace_size(fva_geom g);
 
 /*
@@ -164,9 +165,9 @@ int fva_route_static(const void* qr, const void* kr, fva_geom g, double p, int32
  * fva_route_repair — fva_route followed by fva_repair, fused (same outputs, same
  * arithmetic; the pages describe the two steps, not their split into calls).
  * The per-row repair and compaction run inside fva_route's selection kernel (no
- * mask round trip through memory); one more launch on `stream` builds head_work and
- * the LPT work list.
- *   workspace        : fva_route_workspace_size(g) bytes.
+ * mask round trip through memory); three more launches on `stream` build head_work
+ * and the LPT work list.
+ *   workspace        : fva_route_workspace_size(g) bytes, 256-byte aligned.
  *   topp_mask, topk_idx : as in fva_route, or NULL when the caller does not need them.
  *   counts, idx, head_work, worklist : as in fva_repair (required).
  */
@@ -178,12 +179,16 @@ int fva_route_repair(const void* qr, const void* kr, fva_geom g, double p, int32
 /*
  * fva_route_repair_pooled — fva_route_repair from block means the caller already holds
  * (fva_reorder_pool outputs for Q and K): scoring, Top-p / Top-k selection, repair,
- * W_h and the LPT list, with the same outputs and arithmetic.  No workspace.
+ * W_h and the LPT list, with the same outputs and arithmetic.
  *   qbar, kbar : float64 [B,H,Nb,d], 16-byte aligned.
+ *   workspace  : fva_repair_workspace_size(g) bytes, 256-byte aligned (the LPT sort's
+ *                per-head histograms; nothing in it needs to start at zero).
+ * Four launches: scoring and selection, then the three passes of the LPT sort.
  */
 int fva_route_repair_pooled(const double* qbar, const double* kbar, fva_geom g, double p, int32_t k,
                             uint8_t* topp_mask, int32_t* topk_idx, int32_t* counts, int32_t* idx,
-                            int64_t* head_work, int32_t* worklist, void* stream);
+                            int64_t* head_work, int32_t* worklist, void* workspace, size_t workspace_bytes,
+                            void* stream);
 
 /*
  * fva_route_repair_sasa — fva_route_repair_pooled with slack-aware augmentation, a
@@ -198,7 +203,8 @@ int fva_route_repair_pooled(const double* qbar, const double* kbar, fva_geom g, 
  *   num_ranks : divides H, 1..1024.     alpha : 0..1 (0: no augmentation).
  *   extra     : optional int32 [B,H,Nb] output, the ranked positions added to each row.
  *   workspace : fva_sasa_workspace_size(g) bytes, 256-byte aligned.
- * Four launches: selection, budgets, selection with the extended floors, LPT list.
+ * Six launches: selection, budgets, selection with the extended floors, the three
+ * passes of the LPT sort (its scratch lies in the same workspace).
  */
 size_t fva_sasa_workspace_size(fva_geom g);
 int fva_route_repair_sasa(const double* qbar, const double* kbar, fva_geom g, double p, int32_t k,
@@ -206,7 +212,8 @@ int fva_route_repair_sasa(const double* qbar, const double* kbar, fva_geom g, do
                           int64_t* head_work, int32_t* worklist, int32_t* extra,
                           void* workspace, size_t workspace_bytes, void* stream);
 
-/* Workspace bytes fva_repair needs (currently 0; kept for ABI stability). */
+/* Workspace bytes fva_repair (and fva_route_repair_pooled) need: B*H*(Nb+1) int32 of
+ * per-head count histograms for the LPT sort, rounded up to 256. */
 size_t fva_repair_workspace_size(fva_geom g);
 
 /*
@@ -219,7 +226,10 @@ size_t fva_repair_workspace_size(fva_geom g);
  *   head_work : int64 [B,H] output, W_h = sum over i of counts (kept block pairs).
  *   worklist  : int32 [B*H*Nb] output, item ids u = (b*H + h)*Nb + i ordered by count
  *               descending, ties by u ascending (longest processing time first).
+ *   workspace : fva_repair_workspace_size(g) bytes, 256-byte aligned.
  * Kept set of row i = Top-p set U Top-k floor U {i}.  Requires Nb <= 2048.
+ * The work list is a stable counting sort by count in three passes (per-head
+ * histograms, list offsets, scatter): O(B*H*Nb) work, deterministic.
  */
 int fva_repair(const uint8_t* topp_mask, const int32_t* topk_idx, fva_geom g, int32_t k,
                int32_t* counts, int32_t* idx, int64_t* head_work, int32_t* worklist,
@@ -258,10 +268,24 @@ int fva_block_sparse_attn_natural(const void* qr, const void* kr, const void* vr
 
 /*
  * fva_get_device_error — synchronises `stream`, then reads and clears the device
- * error word that bounded waits inside the kernels set.  *code receives the raw
- * word (0 = none).  Returns FVA_OK, FVA_ERR_TIMEOUT if a wait expired, or FVA_ERR_CUDA.
+ * error word of that stream: the word that kernels this library launched on `stream`
+ * set when a bounded wait expired (1) or an input index was out of range (2).
+ * *code receives the raw word (0 = none).  Each of the first 63 distinct streams used
+ * on a device has its own word; any further stream shares one word with the others
+ * beyond 63.  Returns FVA_OK, FVA_ERR_TIMEOUT if a wait expired, FVA_ERR_INVALID_ARG
+ * for a rejected input, or FVA_ERR_CUDA.
  */
 int fva_get_device_error(void* stream, int32_t* code);
+
+/*
+ * fva_debug_set_wait_limit — TEST ONLY.  Sets the limit, in SM clock cycles, of every
+ * pipeline wait in the attention launches enqueued after this call (process-wide);
+ * cycles <= 0 restores the default (about 2 s).  A test sets a limit far below a
+ * copy's latency so that a wait expires on purpose: the kernel then aborts, waits
+ * for every copy and product it had issued, frees its tensor memory and reports
+ * FVA_ERR_TIMEOUT through fva_get_device_error.  Always returns FVA_OK.
+ */
+int fva_debug_set_wait_limit(int64_t cycles);
 
 /* Thread-local description of the last error returned on this thread ("" if none). */
 const char* fva_last_error(void);

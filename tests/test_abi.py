@@ -43,14 +43,18 @@ def _g(**kw):
 
 def test_workspace_size_queries():
     g = _g()
-    # pooled Q and K (float64), each 256-byte aligned
+    # pooled Q and K (float64), each 256-byte aligned, then the LPT sort's per-head
+    # histograms over the counts 0..Nb (int32)
     nb = g.Nb
     rows = g.B * g.H * nb
     def al(x):
         return (x + 255) // 256 * 256
-    assert fva.fva_route_workspace_size(g) == 2 * al(rows * g.d * 8)
-    assert fva.fva_repair_workspace_size(g) == 0
+    lpt = al(g.B * g.H * (nb + 1) * 4)
+    assert fva.fva_repair_workspace_size(g) == lpt
+    assert fva.fva_route_workspace_size(g) == 2 * al(rows * g.d * 8) + lpt
+    assert fva.fva_sasa_workspace_size(g) == al(2 * ((rows + 63) // 64 * 64) * 4) + lpt
     assert fva.fva_route_workspace_size(_g(X=9)) == 0          # invalid geometry
+    assert fva.fva_repair_workspace_size(_g(X=9)) == 0
 
 
 def _rc(fn, *args):
@@ -93,12 +97,18 @@ def test_invalid_arguments_rejected_on_host():
     assert L.fva_reorder_pool(16, 16, 64, g, None) == fva.FVA_ERR_INVALID_ARG            # in place
     assert L.fva_reorder_pool(16, 32, 68, g, None) == fva.FVA_ERR_INVALID_ARG            # pooled misaligned
     assert L.fva_reorder_pool(16, 32, 64, bad, None) == fva.FVA_ERR_INVALID_ARG
-    pargs = lambda p, k: (256, 512, g, p, k, None, None, 16, 32, 64, 128, None)
+    rneed = fva.fva_repair_workspace_size(_g())
+    assert rneed >= 4 * _g().B * _g().H * (_g().Nb + 1) and rneed % 256 == 0
+    pargs = lambda p, k, ws=4096, wsb=rneed: (256, 512, g, p, k, None, None, 16, 32, 64, 128, ws, wsb, None)
     assert L.fva_route_repair_pooled(*pargs(0.0, 1)) == fva.FVA_ERR_INVALID_ARG
     assert L.fva_route_repair_pooled(*pargs(0.9, 0)) == fva.FVA_ERR_INVALID_ARG
-    assert L.fva_route_repair_pooled(None, 512, g, 0.9, 1, None, None, 16, 32, 64, 128, None) == \
+    assert L.fva_route_repair_pooled(*pargs(0.9, 1, None)) == fva.FVA_ERR_INVALID_ARG       # no workspace
+    assert L.fva_route_repair_pooled(*pargs(0.9, 1, 4096, rneed - 1)) == fva.FVA_ERR_INVALID_ARG
+    assert b"workspace too small" in L.fva_last_error()
+    assert L.fva_route_repair_pooled(*pargs(0.9, 1, 4100)) == fva.FVA_ERR_INVALID_ARG       # not 256-aligned
+    assert L.fva_route_repair_pooled(None, 512, g, 0.9, 1, None, None, 16, 32, 64, 128, 4096, rneed, None) == \
         fva.FVA_ERR_INVALID_ARG
-    assert L.fva_route_repair_pooled(264, 512, g, 0.9, 1, None, None, 16, 32, 64, 128, None) == \
+    assert L.fva_route_repair_pooled(264, 512, g, 0.9, 1, None, None, 16, 32, 64, 128, 4096, rneed, None) == \
         fva.FVA_ERR_INVALID_ARG                                                           # qbar misaligned
     # slack-aware augmentation: num_ranks must divide H, alpha in [0, 1], workspace size
     sneed = fva.fva_sasa_workspace_size(_g())
@@ -110,8 +120,10 @@ def test_invalid_arguments_rejected_on_host():
     assert L.fva_route_repair_sasa(*sargs(2, 0.5, sneed - 1)) == fva.FVA_ERR_INVALID_ARG
     assert sneed >= 2 * 4 * _g().B * _g().H * _g().Nb
     # repair / attention: null pointers, k, unsupported tile for attention
-    assert L.fva_repair(None, 16, g, 1, 16, 16, 16, 16, None, 0, None) == fva.FVA_ERR_INVALID_ARG
-    assert L.fva_repair(16, 16, g, 0, 16, 16, 16, 16, None, 0, None) == fva.FVA_ERR_INVALID_ARG
+    assert L.fva_repair(None, 16, g, 1, 16, 16, 16, 16, 4096, rneed, None) == fva.FVA_ERR_INVALID_ARG
+    assert L.fva_repair(16, 16, g, 0, 16, 16, 16, 16, 4096, rneed, None) == fva.FVA_ERR_INVALID_ARG
+    assert L.fva_repair(16, 16, g, 1, 16, 16, 16, 16, None, 0, None) == fva.FVA_ERR_INVALID_ARG  # no workspace
+    assert L.fva_repair(16, 16, g, 1, 16, 16, 16, 16, 4096, rneed - 4, None) == fva.FVA_ERR_INVALID_ARG
     assert L.fva_block_sparse_attn(16, 16, None, 16, 16, None, g, 0.0, 16, None) == fva.FVA_ERR_INVALID_ARG
     assert L.fva_block_sparse_attn_natural(16, 16, 16, 16, 16, None, g, 0.0, None, None) == fva.FVA_ERR_INVALID_ARG
     assert L.fva_block_sparse_attn_natural(16, 16, 16, 16, 16, None, _g(tt=1, ty=4, tx=8).c(), 0.0, 16, None) == \

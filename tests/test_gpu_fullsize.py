@@ -1,6 +1,7 @@
-"""Full-size parity: the Wan-like 480p and 720p single-layer workloads in the
-launch configuration the benchmark times (LPT work list).  Routing and repair are
-checked in full; attention on a sample of items the oracle computes one by one
+"""Full-size parity: the Wan-like 480p and 720p single-layer workloads, the
+head-heterogeneity stress layer and the 720p layer with 64-token tiles (1200 blocks),
+in the launch configuration the benchmark times (LPT work list).  Routing and repair
+are checked in full; attention on a sample of items the oracle computes one by one
 (the heaviest, the lightest and a seeded random set)."""
 import numpy as np
 import pytest
@@ -21,9 +22,21 @@ def fva():
     return m
 
 
-@pytest.mark.parametrize("name", ["wan480p", "wan720p"])
+FULL = {
+    "wan480p": synth.CONFIGS["wan480p"],
+    "wan720p": synth.CONFIGS["wan720p"],
+    "stress720p": synth.CONFIGS["stress720p"],
+    # the same layer and inputs as wan720p, tiles 1 x 8 x 8
+    "wan720p_tile64": synth.CONFIGS["wan720p"].with_(name="wan720p_tile64", tt=1),
+}
+# share of tie-flagged rows the oracle reports: a row of Nb blocks climbs to p in steps
+# of about 1/Nb of the mass, so wider rows and diffuse heads land in the 1e-5 band more
+TIE_FRAC = {"wan720p_tile64": 0.05, "stress720p": 0.05}
+
+
+@pytest.mark.parametrize("name", list(FULL))
 def test_fullsize(fva, name):
-    cfg = synth.CONFIGS[name]
+    cfg = FULL[name]
     g = fva.Geom.of(cfg)
     og = O.Geometry.of(cfg)
     q, k, v = synth.make_qkv(cfg)
@@ -36,7 +49,7 @@ def test_fullsize(fva, name):
     rr = O.route(qr, kr, og, cfg.p, cfg.k)
     mask_dev = dev["mask"].cpu().numpy()
     topk_dev = dev["topk"].cpu().numpy()
-    n_rows, n_ties, n_diff = check_route(rr, mask_dev, topk_dev)
+    n_rows, n_ties, n_diff = check_route(rr, mask_dev, topk_dev, max_tie_frac=TIE_FRAC.get(name, 0.02))
     print(f"{name}: {n_rows} rows, {n_ties} tie-flagged, {n_diff} differing (all flagged)")
     rp = check_repair(dev, mask_dev, topk_dev)
     density = rp.counts.sum() / (og.B * og.H * og.Nb * og.Nb)

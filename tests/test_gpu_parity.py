@@ -382,3 +382,63 @@ def test_host_pipeline_rejects_device_and_pageable_tensors(fva):
         pipe.submit(pinned, pinned, pinned, torch.zeros(shp, dtype=torch.bfloat16, device="cuda"))
     with pytest.raises(ValueError):
         pipe.submit(pinned, pinned, pinned, torch.zeros((1,) + shp, dtype=torch.bfloat16).pin_memory())
+
+
+def _full_lists(og):
+    """Every key block for every query block (counts Nb, ascending ids)."""
+    Nb = og.Nb
+    counts = np.full((og.B, og.H, Nb), Nb, dtype=np.int32)
+    idx = np.broadcast_to(np.arange(Nb, dtype=np.int32), (og.B, og.H, Nb, Nb)).copy()
+    return counts, idx
+
+
+def test_device_error_word_is_per_stream(fva):
+    """A rejected index raised by a kernel on one stream is reported for that stream only."""
+    cfg = CASES["tiny"]
+    g = fva.Geom.of(cfg)
+    og = O.Geometry.of(cfg)
+    q, k, v = synth.make_qkv(cfg)
+    qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
+    counts, idx = _full_lists(og)
+    bad = idx.copy()
+    bad[0, 1, 2, 0] = og.Nb + 3
+    cd, gd, bd = (torch.from_numpy(a).cuda() for a in (counts, idx, bad))
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    torch.cuda.synchronize()
+    o1, o2 = torch.empty_like(qd), torch.empty_like(qd)
+    fva.fva_block_sparse_attn(qd, kd, vd, cd, bd, None, g, 0.0, o1, stream=s1)
+    fva.fva_block_sparse_attn(qd, kd, vd, cd, gd, None, g, 0.0, o2, stream=s2)
+    assert fva.fva_get_device_error(s2) == 0
+    assert fva.fva_get_device_error(s1) == 2
+    assert fva.fva_get_device_error(s1) == 0
+
+
+def test_wait_expiry_reports_timeout_and_recovers(fva):
+    """With the pipeline wait limit far below a copy's latency every CTA gives up: the
+    call reports FVA_ERR_TIMEOUT (device word 1) after draining its copies and products,
+    and the next call with the default limit on the same stream is correct."""
+    cfg = CASES["d128_s128_multiwave"]
+    g = fva.Geom.of(cfg)
+    og = O.Geometry.of(cfg)
+    q, k, v = synth.make_qkv(cfg)
+    qr, kr, vr = (O.reorder(t, og) for t in (q, k, v))
+    counts, idx = _full_lists(og)
+    args = [to_dev(qr), to_dev(kr), to_dev(vr), torch.from_numpy(counts).cuda(), torch.from_numpy(idx).cuda(), None,
+            g, 0.0]
+    out = torch.zeros((og.B, og.H, og.N, og.d), dtype=torch.bfloat16, device="cuda")
+    torch.cuda.synchronize()
+    fva.fva_debug_set_wait_limit(200)
+    try:
+        fva.fva_block_sparse_attn(*args, out)
+        code = fva.fva_get_device_error()
+    finally:
+        fva.fva_debug_set_wait_limit(0)
+    assert code == 1
+    assert "wait" in fva.fva_last_error()
+    fva.fva_block_sparse_attn(*args, out)
+    assert fva.fva_get_device_error() == 0
+    items = [(b, h, i) for b in range(og.B) for h in range(og.H) for i in (0, og.Nb // 2, og.Nb - 1)]
+    want = O.attention_items(qr, kr, vr, counts, idx, og.S, items)
+    got = bf16_dev_to_f64(out)
+    for (b, h, i), o in want.items():
+        compare_attention(got[b, h, i * og.S:(i + 1) * og.S], o)
