@@ -12,7 +12,7 @@ timed on a bounded sample.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config wan720p] [--impl reference]
                     [--tile-order raster|hilbert] [--static-order] [--no-side-configs]
-                    [--report stress|sweep|sasa]
+                    [--report stress|sweep|sasa|route [--tile64]]
 
 At the default wan720p layer (1 GPU) the line also carries `side_configs`: the
 head-heterogeneity stress layer and the same layer with 64-token tiles, measured
@@ -59,9 +59,10 @@ def parse(argv=None):
     ap.add_argument("--tile-order", choices=("raster", "hilbert"), default="raster",
                     help="tile numbering: raster, or along the 3D Hilbert curve")
     ap.add_argument("--static-order", action="store_true", help="item-id order instead of the LPT work list")
+    ap.add_argument("--tile64", action="store_true", help="--report route: the layer with 1x8x8 tiles")
     ap.add_argument("--no-side-configs", action="store_true",
                     help="skip the stress720p and 64-token-tile keys of the headline line")
-    ap.add_argument("--report", choices=["stress", "sweep", "sasa"], default=None,
+    ap.add_argument("--report", choices=["stress", "sweep", "sasa", "route"], default=None,
                     help="instead of the headline line: head-heterogeneity stress (LPT vs item-id order) or the "
                          "p x tile sweep at 720p scale, one JSON line per measurement")
     return ap.parse_args(argv)
@@ -591,11 +592,57 @@ def run_sasa_report(args):
         print(json.dumps(line), flush=True)
 
 
+def run_route_report(args, reps=5):
+    """Routing calls alone at --config (tile 1x8x8 when the name ends in _tile64): the
+    standalone fva_route_repair from reordered Q and K, its unfused pair and the routing
+    from pooled means, each timed with CUDA events over `reps` calls after one warm-up."""
+    import torch
+    import block_sparse_attention_44_b200 as fva
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream(dev)
+    peaks = load_peaks()
+    name = args.config
+    cfg = synth.CONFIGS[name]
+    if getattr(args, "tile64", False):
+        cfg = cfg.with_(name=name + "_tile64", tt=1)
+    g = fva.Geom.of(cfg)
+    q, k, v = synth.make_qkv(cfg)
+    del v
+    qd, kd = (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev) for a in (q, k))
+    del q, k
+    path = fva.SparseAttention(g, cfg.p, cfg.k, device=dev)
+    fva.fva_reorder_pool(qd, path.qr, path.qbar, g, stream)
+    fva.fva_reorder_pool(kd, path.kr, path.kbar, g, stream)
+    torch.cuda.synchronize()
+    rbytes = 2.0 * g.B * g.H * g.N * g.d * 2
+    calls = {
+        "route_repair": lambda: fva.fva_route_repair(path.qr, path.kr, g, cfg.p, cfg.k, path.rep.counts, path.rep.idx,
+                                                     path.rep.head_work, path.rep.worklist, path.ws, stream=stream),
+        "route": lambda: fva.fva_route(path.qr, path.kr, g, cfg.p, cfg.k, path.route.topp_mask, path.route.topk_idx,
+                                       path.ws, stream=stream),
+        "repair": lambda: fva.fva_repair(path.route.topp_mask, path.route.topk_idx, g, cfg.k, path.rep.counts,
+                                         path.rep.idx, path.rep.head_work, path.rep.worklist, workspace=path.rws,
+                                         stream=stream),
+        "route_repair_pooled": lambda: path.routing(stream),
+    }
+    line = {"report": "route", "workload": workload_desc(cfg)["workload"], "reps": reps}
+    for key, fn in calls.items():
+        line[key + "_ms"] = _time_ms(fn, stream, reps)
+    assert fva.fva_get_device_error(stream) == 0
+    line["routing_gbs"] = rbytes / (line["route_repair_ms"] * 1e-3) / 1e9
+    line["routing_frac_hbm"] = line["routing_gbs"] / peaks["hbm_gbs"]
+    line["density"] = float(path.rep.counts.sum().item()) / (g.B * g.H * g.Nb * g.Nb)
+    print(json.dumps(line), flush=True)
+
+
 def run_report(args):
     import torch
     import block_sparse_attention_44_b200 as fva
     if args.report == "sasa":
         run_sasa_report(args)
+        return
+    if args.report == "route":
+        run_route_report(args)
         return
     dev = torch.device("cuda", 0)
     stream = torch.cuda.current_stream(dev)

@@ -44,9 +44,13 @@ constexpr int kPolyPerEight = 2;
 
 template <int D, int BN, int NSK, int NSV>
 struct AttnCfg {
+  // A "unit" is what one S product covers: KPU kept key blocks of BN rows, KN = 128 key
+  // rows (one block of a 128-token tile, two of a 64-token tile).
+  static constexpr int KPU = kBM / BN;
+  static constexpr int KN = BN * KPU;
   static constexpr int NCH = D / 64;                         // 64-column (128-byte) chunks of a row
   static constexpr int Q_CHUNK = kBM * 128;                  // bytes of one Q chunk (128 rows)
-  static constexpr int KV_CHUNK = BN * 128;                  // bytes of one K or V chunk
+  static constexpr int KV_CHUNK = KN * 128;                  // bytes of one K or V chunk of a unit
   static constexpr int Q_BYTES = NCH * Q_CHUNK;
   static constexpr int KV_BYTES = NCH * KV_CHUNK;
   static constexpr int OFF_Q = 0;
@@ -58,15 +62,15 @@ struct AttnCfg {
   static constexpr int OFF_RED = OFF_BAR + NBAR * 8;         // row maxima / sums [2 parity][2 half][128]
   static constexpr int OFF_MISC = OFF_RED + 2 * 2 * kBM * 4; // tmem base slot, abort flag
   static constexpr int SMEM = OFF_MISC + 16;                 // base must be 1024-aligned (checked)
-  // TMEM columns: S double buffer [0, 2*BN), P double buffer [2*BN, 3*BN) as bf16 pairs
-  // (BN/2 columns each), O after it
-  static constexpr int T_S = 0, T_P = 2 * BN, T_O = 3 * BN;
+  // TMEM columns: S double buffer [0, 2*KN), P double buffer [2*KN, 3*KN) as bf16 pairs
+  // (KN/2 columns each), O after it
+  static constexpr int T_S = 0, T_P = 2 * KN, T_O = 3 * KN;
   static constexpr int TMEM_USED = T_O + D;
   static constexpr int TMEM_COLS = TMEM_USED <= 128 ? 128 : TMEM_USED <= 256 ? 256 : 512;
-  static constexpr uint32_t IDESC_S = idesc_bf16_f32(kBM, BN, false);
+  static constexpr uint32_t IDESC_S = idesc_bf16_f32(kBM, KN, false);
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(kBM, D, true);
   static constexpr uint32_t Q_TX = static_cast<uint32_t>(BN) * D * 2;   // S == BN rows loaded
-  static constexpr uint32_t KV_TX = static_cast<uint32_t>(BN) * D * 2;
+  static constexpr uint32_t KV_TX = static_cast<uint32_t>(KN) * D * 2;
 };
 
 struct AttnParams {
@@ -118,6 +122,8 @@ __device__ __forceinline__ int item_at(const AttnParams& prm, long long it) {
 __device__ __forceinline__ int item_count(const AttnParams& prm, int item) {
   return item < 0 ? 0 : min(prm.counts[item], prm.Nb);
 }
+// Units (S products) of an item with n kept blocks, kpu blocks per unit.
+__device__ __forceinline__ int unit_count(int n, int kpu) { return n <= 0 ? 0 : (n + kpu - 1) / kpu; }
 // Kept key block jj of item `item` (row i), replaced by the diagonal if out of range.
 __device__ __forceinline__ int block_id(const AttnParams& prm, int item, int i, int jj, bool report) {
   int j = prm.idx[static_cast<long long>(item) * prm.Nb + jj];
@@ -128,9 +134,11 @@ __device__ __forceinline__ int block_id(const AttnParams& prm, int item, int i, 
   return j;
 }
 
-// One TMA producer warp: one tile (K or V, 64-column boxes) per kept block through an
-// ns-stage ring; the K producer also loads each item's Q.  The whole warp walks the
-// loop and waits (warp-uniform); lane 0 issues.
+// One TMA producer warp: one ring stage (K or V, 64-column boxes) per unit of KPU kept
+// blocks through an ns-stage ring, the blocks at consecutive row offsets (a unit short
+// of blocks repeats its last block; those rows get probability 0); the K producer also
+// loads each item's Q.  The whole warp walks the loop and waits (warp-uniform); lane 0
+// issues.
 template <int D, int BN, int NS, bool WITH_Q, typename Cfg>
 __device__ void produce(const AttnParams& prm, const CUtensorMap* tm, const CUtensorMap* tmQ, uint32_t ring,
                         uint32_t full0, uint32_t empty0, uint32_t sQ, uint32_t q_full, uint32_t q_empty,
@@ -158,17 +166,22 @@ __device__ void produce(const AttnParams& prm, const CUtensorMap* tm, const CUte
       __syncwarp();
       ++q_items;
     }
-    for (int jj = 0; jj < n; ++jj, ++g) {
+    const int nu = unit_count(n, Cfg::KPU);
+    for (int u = 0; u < nu; ++u, ++g) {
       const int st = static_cast<int>(g % NS);
       if (g >= NS && !(ok = __all_sync(0xffffffffu, mbar_wait(empty0 + 8 * st, ((g / NS) - 1) & 1, abort_flag,
                                                               prm.wait_limit))))
         break;
       if (leader) {
-        const int j = block_id(prm, item, i, jj, WITH_Q);
         mbar_arrive_expect_tx(full0 + 8 * st, Cfg::KV_TX);
-        for (int ch = 0; ch < Cfg::NCH; ++ch)
-          tma_load_2d(ring + st * Cfg::KV_BYTES + ch * Cfg::KV_CHUNK, tm, full0 + 8 * st, ch * 64,
-                      static_cast<int>(row0 + static_cast<long long>(j) * BN));
+#pragma unroll
+        for (int kb = 0; kb < Cfg::KPU; ++kb) {
+          const int jj = min(u * Cfg::KPU + kb, n - 1);
+          const int j = block_id(prm, item, i, jj, WITH_Q && jj == u * Cfg::KPU + kb);
+          for (int ch = 0; ch < Cfg::NCH; ++ch)
+            tma_load_2d(ring + st * Cfg::KV_BYTES + ch * Cfg::KV_CHUNK + kb * BN * 128, tm, full0 + 8 * st, ch * 64,
+                        static_cast<int>(row0 + static_cast<long long>(j) * BN));
+        }
       }
       __syncwarp();
     }
@@ -293,7 +306,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (n <= 0) continue;
       if (!(ok = wait_all(q_full, q_items & 1))) break;
       ++q_items;
-      for (int jj = 0; jj < n; ++jj, ++g) {
+      const int nu = unit_count(n, C::KPU);
+      for (int jj = 0; jj < nu; ++jj, ++g) {
         const int b = static_cast<int>(g & 1);
         const int st = static_cast<int>(g % NSK);
         // S buffer b is free once the softmax has loaded S_{g-2}; the softmax never waits
@@ -304,7 +318,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (leader) {
           tc_fence_after();
           const uint64_t dK = dK0 + static_cast<uint64_t>((st * C::KV_BYTES) >> 4);
-          const uint32_t dS = tmem + C::T_S + b * BN;
+          const uint32_t dS = tmem + C::T_S + b * C::KN;
 #pragma unroll
           for (int ch = 0; ch < C::NCH; ++ch)
 #pragma unroll
@@ -313,7 +327,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                       C::IDESC_S, (ch | kk) != 0);
           umma_commit(k_empty0 + 8 * st);
           umma_commit(s_full0 + 8 * b);
-          if (jj == n - 1) umma_commit(q_empty);   // last reader of this item's Q
+          if (jj == nu - 1) umma_commit(q_empty);   // last reader of this item's Q
         }
         __syncwarp();
         issued = true;
@@ -337,16 +351,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int n = item_count(prm, item);
       if (n <= 0) continue;
       if (items > 0 && !(ok = wait_all(o_free, (items - 1) & 1))) break;   // epilogue read O
-      for (int jj = 0; jj < n; ++jj, ++g) {
+      const int nu = unit_count(n, C::KPU);
+      for (int jj = 0; jj < nu; ++jj, ++g) {
         const int st = static_cast<int>(g % NSV);
         if (!(ok = wait_all(p_full0 + 8 * static_cast<int>(g & 1), (g >> 1) & 1))) break;
         if (!(ok = wait_all(v_full0 + 8 * st, (g / NSV) & 1))) break;
         if (leader) {
           tc_fence_after();
           const uint64_t dV = dV0 + static_cast<uint64_t>((st * C::KV_BYTES) >> 4);
-          const uint32_t aP = tmem + C::T_P + static_cast<uint32_t>(g & 1) * (BN / 2);
+          const uint32_t aP = tmem + C::T_P + static_cast<uint32_t>(g & 1) * (C::KN / 2);
 #pragma unroll
-          for (int ks = 0; ks < BN / 16; ++ks)
+          for (int ks = 0; ks < C::KN / 16; ++ks)
             umma_ts(tmem + C::T_O, aP + ks * 8, dV + ((ks * 16 * 128) >> 4), C::IDESC_PV,
                     (jj > 0 || ks > 0) ? 1u : 0u);
           umma_commit(v_empty0 + 8 * st);
@@ -371,14 +386,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // maxima (and twice per item for the row sums); the barrier also ANDs their
     // "still ok" flags so a bounded-wait failure makes both leave together.  Waits
     // are warp-uniform: the tcgen05.ld/st below are warp-collective.
-    constexpr int HB = BN / 2;                                    // S columns per half
+    constexpr int HB = C::KN / 2;                                 // S columns per half
     constexpr int HD = D / 2;                                     // O columns per half
     const int quarter = warp & 3;
     const int half = (warp - 4) >> 2;
     const int row = quarter * 32 + lane;                          // TMEM lane == query row
+    // with 64-token tiles the lane quarters 2 and 3 hold the zero rows that pad the query
+    // tile to the MMA's 128: their warps skip every load, exponential and store (row r of
+    // P V depends on row r of P only, and those rows of O are never written out)
+    const bool pad = row - lane >= S;
     const int pair_bar = 1 + quarter;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t tP0 = tmem + C::T_P + half * (HB / 2) + lane_off;   // P buffer 0; buffer 1 is BN/2 further
+    const uint32_t tP0 = tmem + C::T_P + half * (HB / 2) + lane_off;   // P buffer 0; buffer 1 is KN/2 further
     const uint32_t tO = tmem + C::T_O + half * HD + lane_off;
     float* red_max = reinterpret_cast<float*>(smem + C::OFF_RED);         // [2][2][kBM]
     const float sl2 = prm.scale_log2;
@@ -410,27 +429,35 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       float m = -INFINITY;   // running max of the scaled logits (base-2 units), same in both halves
       float l = 0.0f;        // this half's running row sum at max m
-      for (int jj = 0; jj < n; ++jj, ++g) {
+      const int nu = unit_count(n, C::KPU);
+      for (int jj = 0; jj < nu; ++jj, ++g) {
         const int b = static_cast<int>(g & 1);
         const int par = b;
+        // a unit short of blocks (the last of an odd count of 64-token blocks) repeats its
+        // last block in the upper half of the key rows: those columns get probability 0
+        const bool dead = pad || (C::KPU == 2 && half == 1 && jj == nu - 1 && (n & 1));
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(s_full0 + 8 * b, (g >> 1) & 1, abort_flag, wlim));
         uint32_t r[HB];
         float pm = -INFINITY;
         if (ok) {
           tc_fence_after();
-          const uint32_t tS = tmem + C::T_S + b * BN + half * HB + lane_off;
+          if (!dead) {
+            const uint32_t tS = tmem + C::T_S + b * C::KN + half * HB + lane_off;
 #pragma unroll
-          for (int c = 0; c < HB / 32; ++c) tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
-          tmem_wait_ld();
+            for (int c = 0; c < HB / 32; ++c) tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
+            tmem_wait_ld();
+          }
           tc_fence_before();
           mbar_arrive(s_free0 + 8 * b);                           // S_j read out: buffer b may be refilled
-          float mx[2] = {-INFINITY, -INFINITY};
+          if (!dead) {
+            float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-          for (int c = 0; c < HB; c += 4) {
-            mx[0] = fmax3(mx[0], __uint_as_float(r[c]), __uint_as_float(r[c + 1]));
-            mx[1] = fmax3(mx[1], __uint_as_float(r[c + 2]), __uint_as_float(r[c + 3]));
+            for (int c = 0; c < HB; c += 4) {
+              mx[0] = fmax3(mx[0], __uint_as_float(r[c]), __uint_as_float(r[c + 1]));
+              mx[1] = fmax3(mx[1], __uint_as_float(r[c + 2]), __uint_as_float(r[c + 3]));
+            }
+            pm = fmaxf(mx[0], mx[1]);
           }
-          pm = fmaxf(mx[0], mx[1]);
           red_max[(par * 2 + half) * kBM + row] = pm;
         }
         ok = bar_and(pair_bar, 64, ok);                           // both halves' maxima published
@@ -443,17 +470,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         const uint64_t negm = f32x2_pack(-m, -m);
         uint64_t rs[4] = {0, 0, 0, 0};      // packed partial row sums
+        if (!dead) {
 #pragma unroll
-        for (int c = 0; c < HB / 2; ++c) {
-          // x = s * scale_log2 - m for two columns at once
-          const uint64_t x2 = ffma2(f32x2_pack(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1])), sl2x2, negm);
-          float x0, x1;
-          f32x2_unpack(x2, x0, x1);
-          const bool poly = (c % 4) < (kPolyPerEight / 2);
-          const float p0 = poly ? exp2_poly(x0) : ex2_approx(x0);
-          const float p1 = poly ? exp2_poly(x1) : ex2_approx(x1);
-          rs[c & 3] = fadd2(rs[c & 3], f32x2_pack(p0, p1));
-          r[c] = pack_bf16x2(p0, p1);
+          for (int c = 0; c < HB / 2; ++c) {
+            // x = s * scale_log2 - m for two columns at once
+            const uint64_t x2 =
+                ffma2(f32x2_pack(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1])), sl2x2, negm);
+            float x0, x1;
+            f32x2_unpack(x2, x0, x1);
+            const bool poly = (c % 4) < (kPolyPerEight / 2);
+            const float p0 = poly ? exp2_poly(x0) : ex2_approx(x0);
+            const float p1 = poly ? exp2_poly(x1) : ex2_approx(x1);
+            rs[c & 3] = fadd2(rs[c & 3], f32x2_pack(p0, p1));
+            r[c] = pack_bf16x2(p0, p1);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < HB / 2; ++c) r[c] = 0u;
         }
         float a0, a1;
         f32x2_unpack(fadd2(fadd2(rs[0], rs[1]), fadd2(rs[2], rs[3])), a0, a1);
@@ -465,14 +498,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (rescale) wait_pv(g - 1);
         if (ok) {
           tc_fence_after();
-          const uint32_t tP = tP0 + static_cast<uint32_t>(b) * (BN / 2);
-          if constexpr (HB / 2 >= 32) {
+          const uint32_t tP = tP0 + static_cast<uint32_t>(b) * (C::KN / 2);
+          if (!pad) {
+            if constexpr (HB / 2 >= 32) {
 #pragma unroll
-            for (int c = 0; c < HB / 64; ++c) tmem_st32(tP + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
-          } else {
-            tmem_st16(tP, r);
+              for (int c = 0; c < HB / 64; ++c) tmem_st32(tP + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
+            } else {
+              tmem_st16(tP, r);
+            }
           }
-          if (rescale) {
+          if (rescale && !pad) {
 #pragma unroll
             for (int c = 0; c < HD / 32; ++c) {
               uint32_t o[32];
@@ -502,7 +537,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (!ok) break;
       tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < HD / 32; ++c) {
+      for (int c = 0; c < (pad ? 0 : HD / 32); ++c) {
         uint32_t o[32];
         tmem_ld32(tO + c * 32, o);
         tmem_wait_ld();
@@ -631,11 +666,11 @@ cudaError_t launch_attention(const void* qr, const void* kr, const void* vr, con
   if (D.d == 128 && D.S == 128)
     e = launch_t<128, 128, 3, 3>(mq, mk, mv, prm, s);
   else if (D.d == 128 && D.S == 64)
-    e = launch_t<128, 64, 5, 5>(mq, mk, mv, prm, s);
+    e = launch_t<128, 64, 3, 3>(mq, mk, mv, prm, s);
   else if (D.d == 64 && D.S == 128)
     e = launch_t<64, 128, 5, 5>(mq, mk, mv, prm, s);
   else
-    e = launch_t<64, 64, 6, 6>(mq, mk, mv, prm, s);
+    e = launch_t<64, 64, 5, 5>(mq, mk, mv, prm, s);
   ++*launches;
   return e;
 }

@@ -50,21 +50,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// try_wait that suspends the thread for at most `ns` nanoseconds (instead of the
-// system-dependent time limit of the plain form).
-__device__ __forceinline__ bool mbar_try_wait_ns(uint32_t bar, uint32_t parity, uint32_t ns) {
+// Non-blocking test of the phase (never suspends the thread).
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}\n"
       : "=r"(ok)
-      : "r"(bar), "r"(parity), "r"(ns)
+      : "r"(bar), "r"(parity)
       : "memory");
   return ok != 0;
 }
-// Limits below this many cycles are test limits: their waits suspend the thread only
-// briefly, so the limit is checked at that resolution.
+// Limits below this many cycles are test limits: their waits poll without suspending
+// (try_wait may suspend the thread for a system-dependent time, longer than such a
+// limit), so the limit is checked at the resolution of one poll.
 constexpr long long kShortWaitLimit = 1000000;
 
 // Waits for phase `parity` of the barrier.  Gives up (returns false) when *abort is
@@ -72,11 +72,10 @@ constexpr long long kShortWaitLimit = 1000000;
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
                                           long long limit = kWaitLimitCycles) {
   const bool short_limit = limit < kShortWaitLimit;
-  const uint32_t ns = static_cast<uint32_t>(short_limit ? (limit / 4 > 0 ? limit / 4 : 1) : 0);
-  if (short_limit ? mbar_try_wait_ns(bar, parity, ns) : mbar_try_wait(bar, parity)) return true;
+  if (short_limit ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
-    if (short_limit ? mbar_try_wait_ns(bar, parity, ns) : mbar_try_wait(bar, parity)) return true;
+    if (short_limit ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
     if (clock64() - t0 > limit) {
       *abort = 1;
@@ -259,6 +258,16 @@ __device__ __forceinline__ bool bar_and(int id, int nthreads, bool pred) {
       : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(nthreads)
       : "memory");
   return r != 0;
+}
+
+// 32 lanes x 16 columns load (half of tmem_ld32).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
 }
 
 // 32 lanes x 16 columns store (half of tmem_st32).

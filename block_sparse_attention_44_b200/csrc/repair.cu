@@ -118,6 +118,7 @@ __global__ void __launch_bounds__(kLptScanThreads) lpt_offsets_kernel(int32_t* _
     tot[e] = 0;
     if (r < V) {
       const int v = V - 1 - r;
+#pragma unroll 8
       for (long long c = 0; c < BH; ++c) tot[e] += hist[c * V + v];
     }
     mine += tot[e];
@@ -141,6 +142,7 @@ __global__ void __launch_bounds__(kLptScanThreads) lpt_offsets_kernel(int32_t* _
     if (r < V) {
       const int v = V - 1 - r;
       long long run = base;
+#pragma unroll 8
       for (long long c = 0; c < BH; ++c) {
         const int n = hist[c * V + v];
         hist[c * V + v] = static_cast<int32_t>(run);
@@ -152,19 +154,23 @@ __global__ void __launch_bounds__(kLptScanThreads) lpt_offsets_kernel(int32_t* _
 }
 
 // grid.x = BH, one warp per CTA.  off: [BH][Nb + 1] first positions from lpt_offsets_kernel.
+// The head's counts are staged in shared memory first (one coalesced pass), so the
+// sequential 32-item steps touch only shared memory and the list.
 __global__ void __launch_bounds__(32) lpt_scatter_kernel(const int32_t* __restrict__ counts, int Nb,
                                                          const int32_t* __restrict__ off,
                                                          int32_t* __restrict__ worklist) {
-  extern __shared__ int cursor[];
+  extern __shared__ int cursor[];        // [Nb + 1] cursors, then [Nb] counts
+  int* cnt = cursor + Nb + 1;
   const long long bh = blockIdx.x;
   const int lane = threadIdx.x;
   for (int v = lane; v <= Nb; v += 32) cursor[v] = off[bh * (Nb + 1) + v];
+  for (int i = lane; i < Nb; i += 32) cnt[i] = lpt_key(__ldg(counts + bh * Nb + i), Nb);
   __syncwarp();
   const unsigned lt = (1u << lane) - 1u;
   for (int i0 = 0; i0 < Nb; i0 += 32) {
     const int i = i0 + lane;
     const bool valid = i < Nb;
-    const int key = valid ? lpt_key(__ldg(counts + bh * Nb + i), Nb) : -1 - lane;   // invalid lanes match no one
+    const int key = valid ? cnt[i] : -1 - lane;   // invalid lanes match no one
     const unsigned peers = __match_any_sync(0xffffffffu, key);
     if (valid) worklist[cursor[key] + __popc(peers & lt)] = static_cast<int32_t>(bh * Nb + i);
     __syncwarp();
@@ -191,7 +197,7 @@ cudaError_t launch_lpt(const int32_t* counts, const Dims& D, int64_t* head_work,
   lpt_offsets_kernel<<<1, kLptScanThreads, 0, s>>>(hist, D.BH(), D.Nb);
   ++*launches;
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  lpt_scatter_kernel<<<grid, 32, hsmem, s>>>(counts, D.Nb, hist, worklist);
+  lpt_scatter_kernel<<<grid, 32, hsmem + static_cast<size_t>(D.Nb) * sizeof(int), s>>>(counts, D.Nb, hist, worklist);
   ++*launches;
   return cudaGetLastError();
 }

@@ -173,6 +173,80 @@ __device__ __forceinline__ unsigned bisect(const unsigned (&q)[PL], const unsign
   return lo;
 }
 
+// Coarse buckets (32 fine buckets each) of the live blocks: kQCap / 32 = 360 of them,
+// held as kHistPerLane per lane.
+constexpr int kHistPerLane = 12;
+constexpr int kHistBins = 32 * kHistPerLane;   // >= kQCap / 32
+static_assert(kHistBins * 32 >= static_cast<int>(kQCap), "histogram covers every live bucket");
+
+// Smallest bucket q (over the live buckets) whose bucket-inclusive mass reaches T, and
+// the mass of every bucket before it.  Requires the total mass to reach T.  Same answer
+// as a bisection over q: the masses are summed per coarse bucket (q >> 5) through a
+// per-warp shared-memory histogram, a warp scan finds the coarse bucket where the
+// running mass reaches T, then a 32-bin histogram of that coarse bucket finds the fine
+// bucket.  `hist` is this warp's kHistBins words of shared memory.
+template <int PL>
+__device__ __forceinline__ unsigned boundary_bucket(const unsigned (&q)[PL], const unsigned (&m)[PL], unsigned T,
+                                                    unsigned* hist, unsigned& above) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int e = 0; e < kHistPerLane; ++e) hist[lane * kHistPerLane + e] = 0u;
+  __syncwarp();
+#pragma unroll
+  for (int s = 0; s < PL; ++s)
+    if (q[s] < kQCap && m[s] != 0u) atomicAdd(&hist[q[s] >> 5], m[s]);
+  __syncwarp();
+  unsigned lane_sum = 0;
+#pragma unroll
+  for (int e = 0; e < kHistPerLane; ++e) lane_sum += hist[lane * kHistPerLane + e];
+  unsigned incl = lane_sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned y = __shfl_up_sync(kFull, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const unsigned excl = incl - lane_sum;
+  // the one lane whose bins take the running mass from below T to T or more
+  const bool mine = excl < T && incl >= T;
+  unsigned bc = 0, before = 0;
+  if (mine) {
+    unsigned pre = excl;
+    for (int e = 0; e < kHistPerLane; ++e) {
+      const unsigned v = hist[lane * kHistPerLane + e];
+      if (pre + v >= T) {
+        bc = static_cast<unsigned>(lane * kHistPerLane + e);
+        before = pre;
+        break;
+      }
+      pre += v;
+    }
+  }
+  const unsigned src = __ffs(__ballot_sync(kFull, mine)) - 1;
+  bc = __shfl_sync(kFull, bc, src);
+  before = __shfl_sync(kFull, before, src);
+  // fine buckets of coarse bucket bc
+  __syncwarp();
+  hist[lane] = 0u;
+  __syncwarp();
+#pragma unroll
+  for (int s = 0; s < PL; ++s)
+    if (q[s] < kQCap && (q[s] >> 5) == bc && m[s] != 0u) atomicAdd(&hist[q[s] & 31u], m[s]);
+  __syncwarp();
+  const unsigned fm = hist[lane];
+  unsigned finc = fm;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned y = __shfl_up_sync(kFull, finc, o);
+    if (lane >= o) finc += y;
+  }
+  const unsigned fexc = before + finc - fm;
+  const bool hit = fexc < T && fexc + fm >= T;
+  const unsigned fsrc = __ffs(__ballot_sync(kFull, hit)) - 1;
+  above = __shfl_sync(kFull, fexc, fsrc);
+  __syncwarp();   // hist is reused by this warp's next row
+  return bc * 32u + fsrc;
+}
+
 // Walks bucket qs in ranking order from weight `acc` (the weight of every better
 // bucket) until the running weight reaches T; returns that block's (key, id).
 // Kr = the row's order keys in shared memory.
@@ -222,7 +296,7 @@ __device__ __forceinline__ bool at_or_before(u64 k, int t, u64 kb, int jb) {
 // Row i of (b, h) = bh; Lr = its logits in shared memory (32*PL entries, -inf past Nb),
 // replaced in place by their order keys once the weights are taken.
 template <int PL>
-__device__ __forceinline__ void select_row(const RouteArgs& a, long long bh, int i, double* Lr) {
+__device__ __forceinline__ void select_row(const RouteArgs& a, long long bh, int i, double* Lr, unsigned* hist) {
   const int lane = threadIdx.x & 31;
   const int Nb = a.Nb;
   const long long row = bh * Nb + i;
@@ -239,7 +313,6 @@ __device__ __forceinline__ void select_row(const RouteArgs& a, long long bh, int
   // more than 45 below the max (weight < e^-45, mass 0) go to bucket kQCap
   unsigned q[PL], m[PL];
   float zl = 0.0f;
-  unsigned qlive = 0;
   u64* Kr = reinterpret_cast<u64*>(Lr);
 #pragma unroll
   for (int s = 0; s < PL; ++s) {
@@ -251,7 +324,6 @@ __device__ __forceinline__ void select_row(const RouteArgs& a, long long bh, int
     zl += e;
     m[s] = __float_as_uint(e);
     q[s] = live ? static_cast<unsigned>(-d * 256.0) : (t < Nb ? kQCap : kQPad);
-    if (live) qlive = max(qlive, q[s]);
     Kr[t] = order_key(L);    // this lane's own slot: no other lane reads it before the swap
   }
   const float z = warp_sum_f32(zl);
@@ -263,7 +335,6 @@ __device__ __forceinline__ void select_row(const RouteArgs& a, long long bh, int
     part += m[s];
   }
   const unsigned tot = __reduce_add_sync(kFull, part);
-  qlive = __reduce_max_sync(kFull, qlive);
 
   // Top-p boundary (kpb, jpb): the kept set is every block ranking at or before it
   const bool all_p = a.keep_all_p || tot < a.target;
@@ -271,24 +342,41 @@ __device__ __forceinline__ void select_row(const RouteArgs& a, long long bh, int
   u64 kpb = 0;
   int jpb = INT_MAX;
   if (!all_p) {
-    qp = bisect<PL, true>(q, m, 0u, qlive, a.target);
     unsigned above = 0;
-#pragma unroll
-    for (int s = 0; s < PL; ++s)
-      if (q[s] < qp) above += m[s];
-    above = __reduce_add_sync(kFull, above);
+    qp = boundary_bucket<PL>(q, m, a.target, hist, above);
     walk_bucket<PL, true>(Kr, q, m, qp, above, a.target, kpb, jpb);
   }
 
-  // Top-k floor: bit s of `taken` marks block lane + 32 s (kk <= kTopkArgmaxMax)
+  // Top-p membership bits of this lane's blocks and the set's size n_p
+  unsigned long long inp = 0;
+#pragma unroll
+  for (int s = 0; s < PL; ++s) {
+    const int t = lane + 32 * s;
+    bool in = all_p || q[s] < qp;
+    if (!all_p && q[s] == qp) in = at_or_before(Kr[t], t, kpb, jpb);
+    if (in && t < Nb) inp |= 1ull << s;
+  }
+  unsigned np_lane = 0;
+#pragma unroll
+  for (int s = 0; s < PL; ++s) np_lane += static_cast<unsigned>((inp >> s) & 1ull);
+  const int n_p = static_cast<int>(__reduce_add_sync(kFull, np_lane));
+
+  // Top-k floor: bit s of `taken` marks block lane + 32 s (kk <= kTopkArgmaxMax).  Both the
+  // floor and the Top-p set are prefixes of the same ranking, so when the Top-p set holds
+  // at least kk blocks the floor adds nothing to the kept set and is skipped unless its
+  // ids are an output.
   const int kk = a.kk_rows ? a.kk_rows[row] : a.kk;
+  int32_t* krow = a.topk_idx ? a.topk_idx + row * kk : nullptr;
+  const bool need_floor = krow != nullptr || n_p < kk;
   unsigned long long taken = 0;
   unsigned qk = 0;
   u64 kkb = 0;
   int jkb = INT_MAX;
-  int32_t* krow = a.topk_idx ? a.topk_idx + row * kk : nullptr;
   unsigned mine = 0xFFFFFFFFu;   // lane c holds the c-th chosen id
-  if (kk <= 4) {
+  const bool big_k = kk > kTopkArgmaxMax;
+  if (!need_floor) {
+    // kept set = Top-p set (plus the diagonal)
+  } else if (kk <= 4) {
     // each lane's four best (key descending, id ascending) in one pass, then four
     // warp-wide picks among the lane heads
     u64 k4[4] = {0, 0, 0, 0};
@@ -322,7 +410,7 @@ __device__ __forceinline__ void select_row(const RouteArgs& a, long long bh, int
       }
       if (lane == c) mine = wt;
     }
-  } else if (kk <= kTopkArgmaxMax) {
+  } else if (!big_k) {
     for (int c = 0; c < kk; ++c) {
       u64 bk = 0;
       unsigned bt = 0xFFFFFFFFu;
@@ -351,31 +439,23 @@ __device__ __forceinline__ void select_row(const RouteArgs& a, long long bh, int
     above = __reduce_add_sync(kFull, above);
     walk_bucket<PL, false>(Kr, q, m, qk, above, static_cast<unsigned>(kk), kkb, jkb);
   }
-  const bool big_k = kk > kTopkArgmaxMax;
   if (krow && !big_k) {   // ascending block id: lane c writes its id at its rank
     int rank = 0;
     for (int c = 0; c < kk; ++c) rank += __shfl_sync(kFull, mine, c) < mine ? 1 : 0;
     if (lane < kk) krow[rank] = static_cast<int32_t>(mine);
   }
 
-  // membership bits of this lane's blocks: Top-p set, floor
-  unsigned long long inp = 0, ink = taken;
+  // floor membership bits (large floors)
+  unsigned long long ink = taken;
+  if (need_floor && big_k) {
 #pragma unroll
-  for (int s = 0; s < PL; ++s) {
-    const int t = lane + 32 * s;
-    bool in = all_p || q[s] < qp;
-    if (!all_p && q[s] == qp) in = at_or_before(Kr[t], t, kpb, jpb);
-    if (in && t < Nb) inp |= 1ull << s;
-    if (big_k && t < Nb && (q[s] < qk || (q[s] == qk && at_or_before(Kr[t], t, kkb, jkb)))) ink |= 1ull << s;
+    for (int s = 0; s < PL; ++s) {
+      const int t = lane + 32 * s;
+      if (t < Nb && (q[s] < qk || (q[s] == qk && at_or_before(Kr[t], t, kkb, jkb)))) ink |= 1ull << s;
+    }
   }
 
-  if (a.prefix_out) {   // n_p = size of the Top-p set
-    unsigned np_lane = 0;
-#pragma unroll
-    for (int s = 0; s < PL; ++s) np_lane += static_cast<unsigned>((inp >> s) & 1ull);
-    const int n_p = static_cast<int>(__reduce_add_sync(kFull, np_lane));
-    if (lane == 0) a.prefix_out[row] = n_p > kk ? n_p : kk;
-  }
+  if (a.prefix_out && lane == 0) a.prefix_out[row] = n_p > kk ? n_p : kk;   // length of the kept ranked prefix
 
   // outputs: compacted kept list, Top-p mask, floor ids (large floors), logits
   const int nsl = (Nb + 31) / 32;   // slots holding blocks
@@ -428,6 +508,7 @@ __device__ __forceinline__ void select_item(const RouteArgs& a, long long bh, in
   constexpr int NT = 4 * PL;             // 8-column tiles covering 32 * PL columns
   double* Qs = reinterpret_cast<double*>(smem);
   double* Ls = Qs + R * LDQ;
+  unsigned* Hs = reinterpret_cast<unsigned*>(Ls + R * LDL);   // per-warp histograms
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int Nb = a.Nb;
 
@@ -503,12 +584,13 @@ __device__ __forceinline__ void select_item(const RouteArgs& a, long long bh, in
   __syncthreads();
 
   for (int r = warp; r < R; r += kRouteWarps)
-    if (i0 + r < Nb) select_row<PL>(a, bh, i0 + r, Ls + r * LDL);
+    if (i0 + r < Nb) select_row<PL>(a, bh, i0 + r, Ls + r * LDL, Hs + warp * kHistBins);
 }
 
 template <int D, int PL, int R>
 constexpr size_t select_smem_bytes() {
-  return (static_cast<size_t>(R) * (D + 4) + static_cast<size_t>(R) * (32 * PL + 2)) * sizeof(double);
+  return (static_cast<size_t>(R) * (D + 4) + static_cast<size_t>(R) * (32 * PL + 2)) * sizeof(double) +
+         static_cast<size_t>(kRouteWarps) * kHistBins * sizeof(unsigned);
 }
 
 // grid = (ceil(Nb / R), heads): CTA (x, y) selects rows [x*R, x*R + R) of (b, h) = bh0 + y.

@@ -431,10 +431,11 @@ def test_wait_expiry_reports_timeout_and_recovers(fva):
     try:
         fva.fva_block_sparse_attn(*args, out)
         code = fva.fva_get_device_error()
+        msg = fva.fva_last_error()
     finally:
         fva.fva_debug_set_wait_limit(0)
     assert code == 1
-    assert "wait" in fva.fva_last_error()
+    assert "wait" in msg
     fva.fva_block_sparse_attn(*args, out)
     assert fva.fva_get_device_error() == 0
     items = [(b, h, i) for b in range(og.B) for h in range(og.H) for i in (0, og.Nb // 2, og.Nb - 1)]
