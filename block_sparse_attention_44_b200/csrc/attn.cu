@@ -41,6 +41,13 @@ constexpr float kLazyRescaleLog2 = 8.0f;
 // Of every 8 probabilities a softmax thread computes, this many use the FMA-pipe
 // exp2 (exp2_poly) instead of the MUFU unit, so both units share the work.
 constexpr int kPolyPerEight = 2;
+// Register split between the control warpgroup (warps 0-3) and the two softmax warpgroups.
+constexpr int kCtrlRegs = 80;
+constexpr int kSoftmaxRegs = 192;
+// Bitmap words of one kept list (one bit per key block, up to kMaxNb blocks).
+constexpr int kBmWords = kMaxNb / 32;
+// Warps that copy the pair bitmaps (all but the K producer, which builds them).
+constexpr int kBmReaders = kAttnThreads / 32 - 1;
 
 template <int D, int BN, int NSK, int NSV>
 struct AttnCfg {
@@ -57,11 +64,13 @@ struct AttnCfg {
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
   static constexpr int OFF_V = OFF_K + NSK * KV_BYTES;
   static constexpr int OFF_BAR = OFF_V + NSV * KV_BYTES;
-  // barriers: q_full q_empty s_full[2] s_free[2] p_full[2] o_done[2] o_free drain_s drain_pv; k ring; v ring
-  static constexpr int NBAR = 13 + 2 * NSK + 2 * NSV;
+  // barriers: q_full q_empty s_full[2] s_free[2] p_full[2] o_done[2] o_free drain_s drain_pv bm_full
+  // bm_empty; k ring; v ring
+  static constexpr int NBAR = 15 + 2 * NSK + 2 * NSV;
   static constexpr int OFF_RED = OFF_BAR + NBAR * 8;         // row maxima / sums [2 parity][2 half][128]
   static constexpr int OFF_MISC = OFF_RED + 2 * 2 * kBM * 4; // tmem base slot, abort flag
-  static constexpr int SMEM = OFF_MISC + 16;                 // base must be 1024-aligned (checked)
+  static constexpr int OFF_BM = OFF_MISC + 16;               // kept-block bitmaps of a query-block pair
+  static constexpr int SMEM = OFF_BM + 2 * kBmWords * 4;     // base must be 1024-aligned (checked)
   // TMEM columns: S double buffer [0, 2*KN), P double buffer [2*KN, 3*KN) as bf16 pairs
   // (KN/2 columns each), O after it
   static constexpr int T_S = 0, T_P = 2 * KN, T_O = 3 * KN;
@@ -122,7 +131,70 @@ __device__ __forceinline__ int item_at(const AttnParams& prm, long long it) {
 __device__ __forceinline__ int item_count(const AttnParams& prm, int item) {
   return item < 0 ? 0 : min(prm.counts[item], prm.Nb);
 }
-// Units (S products) of an item with n kept blocks, kpu blocks per unit.
+// One work item of the kernel.  With 128-token tiles: one query block (item).  With 64-token
+// tiles: two adjacent query blocks 2p and 2p + 1 of a head share the 128-row query tile (rows
+// 0-63 and 64-127) and run over the union of their kept lists, two key blocks per S product;
+// each row masks the keys outside its own block's list, so every row's result is that of
+// its own list.  The work list's entries for odd blocks are skipped (their pair is processed
+// at the entry of the even block).
+struct Work {
+  int item;     // item id of the (first) query block
+  int nq;       // query blocks in the tile (2 for a full pair)
+  int n0, n1;   // kept-list lengths of the two blocks (n1 = 0 without a second block)
+};
+template <int KPU>
+__device__ __forceinline__ bool work_at(const AttnParams& prm, long long it, Work& w) {
+  const int item = item_at(prm, it);
+  if (item < 0) return false;
+  w.item = item;
+  w.n0 = item_count(prm, item);
+  if (KPU == 1) {
+    w.nq = 1;
+    w.n1 = 0;
+    return true;
+  }
+  const int i = item % prm.Nb;
+  if (i & 1) return false;
+  w.nq = i + 1 < prm.Nb ? 2 : 1;
+  w.n1 = w.nq == 2 ? item_count(prm, item + 1) : 0;
+  return true;
+}
+
+// Union of a pair's two kept-list bitmaps held across a warp's lanes (lane l: words l and
+// l + 32), walked in ascending block order; every role walks it the same way.
+struct Bitmaps {
+  uint32_t a0, a1, b0, b1;   // this lane's words of block 2p's and block 2p+1's lists
+};
+__device__ __forceinline__ Bitmaps load_bitmaps(const uint32_t* bm) {
+  const int lane = threadIdx.x & 31;
+  return Bitmaps{bm[lane], bm[lane + 32], bm[kBmWords + lane], bm[kBmWords + lane + 32]};
+}
+__device__ __forceinline__ int union_size(const Bitmaps& b) {
+  return static_cast<int>(__reduce_add_sync(0xffffffffu, __popc(b.a0 | b.b0) + __popc(b.a1 | b.b1)));
+}
+// Next key block of the union (warp-uniform cursor; -1 when exhausted).
+struct Cursor {
+  int w = -1;
+  uint32_t rb = 0;
+};
+__device__ __forceinline__ int next_key(Cursor& c, const Bitmaps& b, int nwords) {
+  while (c.rb == 0) {
+    if (++c.w >= nwords) return -1;
+    const uint32_t lo = b.a0 | b.b0, hi = b.a1 | b.b1;
+    c.rb = __shfl_sync(0xffffffffu, c.w < 32 ? lo : hi, c.w & 31);
+  }
+  const int j = c.w * 32 + __ffs(c.rb) - 1;
+  c.rb &= c.rb - 1;
+  return j;
+}
+// Whether key block j is in the list of the pair's block `which` (0 or 1); warp-uniform.
+__device__ __forceinline__ bool in_list(const Bitmaps& b, int which, int j) {
+  const int w = j >> 5;
+  const uint32_t lo = which ? b.b0 : b.a0, hi = which ? b.b1 : b.a1;
+  return (__shfl_sync(0xffffffffu, w < 32 ? lo : hi, w & 31) >> (j & 31)) & 1u;
+}
+// Units (S products) of a work item: its kept blocks with 128-token tiles; half the union
+// of the two lists, rounded up, with 64-token tiles.
 __device__ __forceinline__ int unit_count(int n, int kpu) { return n <= 0 ? 0 : (n + kpu - 1) / kpu; }
 // Kept key block jj of item `item` (row i), replaced by the diagonal if out of range.
 __device__ __forceinline__ int block_id(const AttnParams& prm, int item, int i, int jj, bool report) {
@@ -134,40 +206,88 @@ __device__ __forceinline__ int block_id(const AttnParams& prm, int item, int i, 
   return j;
 }
 
-// One TMA producer warp: one ring stage (K or V, 64-column boxes) per unit of KPU kept
-// blocks through an ns-stage ring, the blocks at consecutive row offsets (a unit short
-// of blocks repeats its last block; those rows get probability 0); the K producer also
-// loads each item's Q.  The whole warp walks the loop and waits (warp-uniform); lane 0
-// issues.
+// Bitmaps of a work item for the warps that read them: the K producer builds them (below);
+// every other warp waits for them, copies its lanes' words and releases the buffer.
+__device__ __forceinline__ bool copy_bitmaps(const uint32_t* bm, uint32_t bm_full, uint32_t bm_empty, long long k,
+                                             volatile int* abort_flag, long long wlim, Bitmaps& out) {
+  if (!__all_sync(0xffffffffu, mbar_wait(bm_full, k & 1, abort_flag, wlim))) return false;
+  out = load_bitmaps(bm);
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bm_empty);
+  return true;
+}
+
+// One TMA producer warp: one ring stage (K or V, 64-column boxes) per unit of KPU key blocks
+// through an ns-stage ring, the blocks at consecutive row offsets.  With 64-token tiles the
+// unit's two key blocks are the next two of the pair's union (a unit short of a block repeats
+// its block; those rows get probability 0).  The K producer also loads each work item's Q
+// rows and, with 64-token tiles, builds the pair's kept-list bitmaps.  The whole warp walks
+// the loop and waits (warp-uniform); lane 0 issues.
 template <int D, int BN, int NS, bool WITH_Q, typename Cfg>
 __device__ void produce(const AttnParams& prm, const CUtensorMap* tm, const CUtensorMap* tmQ, uint32_t ring,
                         uint32_t full0, uint32_t empty0, uint32_t sQ, uint32_t q_full, uint32_t q_empty,
-                        volatile int* abort_flag) {
+                        uint32_t* bm, uint32_t bm_full, uint32_t bm_empty, volatile int* abort_flag) {
   const int Nb = prm.Nb;
-  const bool leader = (threadIdx.x & 31) == 0;
-  long long g = 0, q_items = 0;
+  const int lane = threadIdx.x & 31;
+  const bool leader = lane == 0;
+  const int nwords = (Nb + 31) / 32;
+  long long g = 0, q_items = 0, pairs = 0;
   bool ok = true;
   for (long long it = blockIdx.x; it < prm.n_items && ok; it += gridDim.x) {
-    const int item = item_at(prm, it);
-    const int n = item_count(prm, item);
-    if (n <= 0) continue;
-    const long long bh = item / Nb;
-    const int i = item - static_cast<int>(bh * Nb);
+    Work w;
+    if (!work_at<Cfg::KPU>(prm, it, w) || w.n0 + w.n1 <= 0) continue;
+    const long long bh = w.item / Nb;
+    const int i = w.item - static_cast<int>(bh * Nb);
     const long long row0 = bh * prm.N;
+    Bitmaps bmr{0, 0, 0, 0};
+    int nu = w.n0;
+    if (Cfg::KPU == 2) {
+      if (WITH_Q) {
+        // every reader has copied the previous pair's bitmaps
+        if (pairs > 0 &&
+            !(ok = __all_sync(0xffffffffu, mbar_wait(bm_empty, (pairs - 1) & 1, abort_flag, prm.wait_limit))))
+          break;
+        for (int e = lane; e < 2 * kBmWords; e += 32) bm[e] = 0u;
+        __syncwarp();
+        for (int x = 0; x < w.nq; ++x) {
+          const int n = x ? w.n1 : w.n0;
+          for (int c = lane; c < n; c += 32) {
+            const int j = block_id(prm, w.item + x, i + x, c, true);
+            atomicOr(&bm[x * kBmWords + (j >> 5)], 1u << (j & 31));
+          }
+        }
+        __threadfence_block();
+        __syncwarp();
+        if (leader) mbar_arrive(bm_full);
+        bmr = load_bitmaps(bm);
+      } else if (!(ok = copy_bitmaps(bm, bm_full, bm_empty, pairs, abort_flag, prm.wait_limit, bmr))) {
+        break;
+      }
+      ++pairs;
+      nu = (union_size(bmr) + 1) / 2;
+    }
     if (WITH_Q) {
       if (q_items > 0 &&
           !(ok = __all_sync(0xffffffffu, mbar_wait(q_empty, (q_items - 1) & 1, abort_flag, prm.wait_limit))))
         break;
       if (leader) {
-        mbar_arrive_expect_tx(q_full, Cfg::Q_TX);
-        for (int ch = 0; ch < Cfg::NCH; ++ch)
-          tma_load_2d(sQ + ch * Cfg::Q_CHUNK, tmQ, q_full, ch * 64, static_cast<int>(row0 + static_cast<long long>(i) * BN));
+        mbar_arrive_expect_tx(q_full, Cfg::Q_TX * static_cast<uint32_t>(w.nq));
+        for (int x = 0; x < w.nq; ++x)
+          for (int ch = 0; ch < Cfg::NCH; ++ch)
+            tma_load_2d(sQ + ch * Cfg::Q_CHUNK + x * BN * 128, tmQ, q_full, ch * 64,
+                        static_cast<int>(row0 + static_cast<long long>(i + x) * BN));
       }
       __syncwarp();
       ++q_items;
     }
-    const int nu = unit_count(n, Cfg::KPU);
+    Cursor cur;
     for (int u = 0; u < nu; ++u, ++g) {
+      int j0 = 0, j1 = 0;
+      if (Cfg::KPU == 2) {
+        j0 = next_key(cur, bmr, nwords);
+        j1 = next_key(cur, bmr, nwords);
+        if (j1 < 0) j1 = j0;
+      }
       const int st = static_cast<int>(g % NS);
       if (g >= NS && !(ok = __all_sync(0xffffffffu, mbar_wait(empty0 + 8 * st, ((g / NS) - 1) & 1, abort_flag,
                                                               prm.wait_limit))))
@@ -176,8 +296,7 @@ __device__ void produce(const AttnParams& prm, const CUtensorMap* tm, const CUte
         mbar_arrive_expect_tx(full0 + 8 * st, Cfg::KV_TX);
 #pragma unroll
         for (int kb = 0; kb < Cfg::KPU; ++kb) {
-          const int jj = min(u * Cfg::KPU + kb, n - 1);
-          const int j = block_id(prm, item, i, jj, WITH_Q && jj == u * Cfg::KPU + kb);
+          const int j = Cfg::KPU == 1 ? block_id(prm, w.item, i, u, WITH_Q) : (kb ? j1 : j0);
           for (int ch = 0; ch < Cfg::NCH; ++ch)
             tma_load_2d(ring + st * Cfg::KV_BYTES + ch * Cfg::KV_CHUNK + kb * BN * 128, tm, full0 + 8 * st, ch * 64,
                         static_cast<int>(row0 + static_cast<long long>(j) * BN));
@@ -216,13 +335,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t bar0 = sbase + C::OFF_BAR;
   const uint32_t q_full = bar0, q_empty = bar0 + 8, s_full0 = bar0 + 16, s_free0 = bar0 + 32;
   const uint32_t p_full0 = bar0 + 48, o_done0 = bar0 + 64, o_free = bar0 + 80, drain_s = bar0 + 88;
-  const uint32_t drain_pv = bar0 + 96;
-  const uint32_t k_full0 = bar0 + 104;
+  const uint32_t drain_pv = bar0 + 96, bm_full = bar0 + 104, bm_empty = bar0 + 112;
+  const uint32_t k_full0 = bar0 + 120;
   const uint32_t k_empty0 = k_full0 + 8 * NSK;
   const uint32_t v_full0 = k_empty0 + 8 * NSK;
   const uint32_t v_empty0 = v_full0 + 8 * NSV;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  uint32_t* bm = reinterpret_cast<uint32_t*>(smem + C::OFF_BM);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x & 31;
@@ -239,6 +359,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     mbar_init(o_free, 256);
     mbar_init(drain_s, 1);
     mbar_init(drain_pv, 1);
+    mbar_init(bm_full, 1);
+    mbar_init(bm_empty, kBmReaders);
     for (int st = 0; st < NSK; ++st) {
       mbar_init(k_full0 + 8 * st, 1);
       mbar_init(k_empty0 + 8 * st, 1);
@@ -281,12 +403,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, wlim));
   };
 
+  // Registers: the launch gives every thread 168; the control warpgroup returns what it
+  // does not need and the softmax warpgroups take it.  128 x kCtrlRegs + 256 x kSoftmaxRegs
+  // stays within the launch's 384 x 168, so the increase always finds its registers.
+  static_assert(128 * kCtrlRegs + 256 * kSoftmaxRegs <= kAttnThreads * 168, "register split exceeds the launch");
+  if (warp < 4) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtrlRegs));
   if (warp == 0) {
     // ---------------------------------------------------------------- Q + K producer
-    produce<D, BN, NSK, true, C>(prm, &tmK, &tmQ, sK, k_full0, k_empty0, sQ, q_full, q_empty, abort_flag);
+    produce<D, BN, NSK, true, C>(prm, &tmK, &tmQ, sK, k_full0, k_empty0, sQ, q_full, q_empty, bm, bm_full, bm_empty,
+                                 abort_flag);
   } else if (warp == 3) {
     // ---------------------------------------------------------------- V producer
-    produce<D, BN, NSV, false, C>(prm, &tmV, &tmQ, sV, v_full0, v_empty0, sQ, q_full, q_empty, abort_flag);
+    produce<D, BN, NSV, false, C>(prm, &tmV, &tmQ, sV, v_full0, v_empty0, sQ, q_full, q_empty, bm, bm_full, bm_empty,
+                                  abort_flag);
   } else if (warp == 1) {
     // ---------------------------------------------------------------- S issuer
     // S_j = Q K_j^T into S buffer j % 2 as soon as the softmax has read S_{j-2} out of it.
@@ -298,15 +428,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint64_t dK0 = sdesc_sw128(sK, 16, 1024);
     // (descriptor start addresses are the low 14 bits, address >> 4; operands lie
     //  below 256 KB, so byte offsets add in without carry)
-    long long g = 0, q_items = 0;
+    long long g = 0, q_items = 0, pairs = 0;
     bool ok = true, issued = false;
     for (long long it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-      const int item = item_at(prm, it);
-      const int n = item_count(prm, item);
-      if (n <= 0) continue;
+      Work w;
+      if (!work_at<C::KPU>(prm, it, w) || w.n0 + w.n1 <= 0) continue;
       if (!(ok = wait_all(q_full, q_items & 1))) break;
       ++q_items;
-      const int nu = unit_count(n, C::KPU);
+      int nu = w.n0;
+      if (C::KPU == 2) {
+        Bitmaps bmr;
+        if (!(ok = copy_bitmaps(bm, bm_full, bm_empty, pairs++, abort_flag, wlim, bmr))) break;
+        nu = (union_size(bmr) + 1) / 2;
+      }
       for (int jj = 0; jj < nu; ++jj, ++g) {
         const int b = static_cast<int>(g & 1);
         const int st = static_cast<int>(g % NSK);
@@ -344,14 +478,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // O += P_j V_j once the softmax has written P_j into P buffer j % 2 (p_full); the
     // commit on o_done[j % 2] tells the softmax that buffer and O are free again.
     const uint64_t dV0 = sdesc_sw128(sV, C::KV_CHUNK, 1024);
-    long long g = 0, items = 0;
+    long long g = 0, items = 0, pairs = 0;
     bool ok = true, issued = false;
     for (long long it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-      const int item = item_at(prm, it);
-      const int n = item_count(prm, item);
-      if (n <= 0) continue;
+      Work w;
+      if (!work_at<C::KPU>(prm, it, w) || w.n0 + w.n1 <= 0) continue;
+      int nu = w.n0;
+      if (C::KPU == 2) {
+        Bitmaps bmr;
+        if (!(ok = copy_bitmaps(bm, bm_full, bm_empty, pairs++, abort_flag, wlim, bmr))) break;
+        nu = (union_size(bmr) + 1) / 2;
+      }
       if (items > 0 && !(ok = wait_all(o_free, (items - 1) & 1))) break;   // epilogue read O
-      const int nu = unit_count(n, C::KPU);
       for (int jj = 0; jj < nu; ++jj, ++g) {
         const int st = static_cast<int>(g % NSV);
         if (!(ok = wait_all(p_full0 + 8 * static_cast<int>(g & 1), (g >> 1) & 1))) break;
@@ -378,7 +516,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       __syncwarp();
       drain_wait(drain_pv, 0);
     }
-  } else if (warp >= 4) {
+  }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
     // ---------------------------------------------------------------- softmax
     // Eight warps: warp w owns TMEM lane quarter w % 4 (query rows 32*(w%4) ...) and
     // half h = (w - 4) / 4 of the columns of S (and of P and O).  The two warps of a
@@ -391,10 +531,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int quarter = warp & 3;
     const int half = (warp - 4) >> 2;
     const int row = quarter * 32 + lane;                          // TMEM lane == query row
-    // with 64-token tiles the lane quarters 2 and 3 hold the zero rows that pad the query
-    // tile to the MMA's 128: their warps skip every load, exponential and store (row r of
-    // P V depends on row r of P only, and those rows of O are never written out)
-    const bool pad = row - lane >= S;
+    // query block of this warp's rows within the work item: with 64-token tiles lane
+    // quarters 0-1 hold block 2p and quarters 2-3 block 2p + 1
+    const int which = C::KPU == 2 ? quarter >> 1 : 0;
+    const int rloc = row - which * S;                             // row within its query block
+    const int nwords = (Nb + 31) / 32;
     const int pair_bar = 1 + quarter;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t tP0 = tmem + C::T_P + half * (HB / 2) + lane_off;   // P buffer 0; buffer 1 is KN/2 further
@@ -402,7 +543,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     float* red_max = reinterpret_cast<float*>(smem + C::OFF_RED);         // [2][2][kBM]
     const float sl2 = prm.scale_log2;
     const uint64_t sl2x2 = f32x2_pack(sl2, sl2);
-    long long g = 0;   // blocks processed
+    long long g = 0, pairs = 0;   // units processed; pairs whose bitmaps were copied
     bool ok = true;
     // wait until P_q V_q has completed (its commit on o_done[q % 2] is that barrier's
     // phase q / 2; P_{q+2} V_{q+2} cannot start before this warp writes P_{q+2}, so the
@@ -413,29 +554,46 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                                                wlim));
     };
     for (long long it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-      const int item = item_at(prm, it);
-      if (item < 0) continue;
-      const int n = item_count(prm, item);
-      const long long bh = item / Nb;
-      const int i = item - static_cast<int>(bh * Nb);
-      const long long tok = out_token(prm, i, row < S ? row : 0, S);
+      Work w;
+      if (!work_at<C::KPU>(prm, it, w)) continue;
+      const long long bh = w.item / Nb;
+      const int i = w.item - static_cast<int>(bh * Nb);
+      // rows of a query block the tile does not hold (64-token tiles: the odd last block of a
+      // head has no partner) skip every load, exponential and store: row r of P V depends on
+      // row r of P only, and those rows of O are never written out
+      const bool pad = which >= w.nq;
+      const int nrow = which ? w.n1 : w.n0;                       // kept blocks of this row's block
+      const long long tok = pad ? 0 : out_token(prm, i + which, rloc < S ? rloc : 0, S);
       if (tok < 0) set_device_error(prm.dev_err, kDevErrBadIndex);
       uint16_t* orow = prm.out + (bh * prm.N + (tok < 0 ? 0 : tok)) * D + half * HD;
-      const bool wr = row < S && tok >= 0;   // this thread writes its row
-      if (n <= 0) {
+      const bool wr = !pad && rloc < S && tok >= 0;   // this thread writes its row
+      if (w.n0 + w.n1 <= 0) {
         if (wr)
           for (int c = 0; c < HD; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
         continue;
       }
+      Bitmaps bmr{0, 0, 0, 0};
+      int nu = w.n0;
+      if (C::KPU == 2) {
+        if (!(ok = copy_bitmaps(bm, bm_full, bm_empty, pairs++, abort_flag, wlim, bmr))) break;
+        nu = (union_size(bmr) + 1) / 2;
+      }
+      Cursor cur;
       float m = -INFINITY;   // running max of the scaled logits (base-2 units), same in both halves
       float l = 0.0f;        // this half's running row sum at max m
-      const int nu = unit_count(n, C::KPU);
       for (int jj = 0; jj < nu; ++jj, ++g) {
         const int b = static_cast<int>(g & 1);
         const int par = b;
-        // a unit short of blocks (the last of an odd count of 64-token blocks) repeats its
-        // last block in the upper half of the key rows: those columns get probability 0
-        const bool dead = pad || (C::KPU == 2 && half == 1 && jj == nu - 1 && (n & 1));
+        // this half's key block: the unit's block with 128-token tiles; with 64-token tiles
+        // the unit's first or second union block, dead (probability 0) when it is missing or
+        // outside this row's own kept list
+        bool dead = pad || nrow <= 0;
+        if (C::KPU == 2) {
+          const int j0 = next_key(cur, bmr, nwords);
+          const int j1 = next_key(cur, bmr, nwords);
+          const int key = half ? j1 : j0;
+          dead = dead || key < 0 || !in_list(bmr, which, key);
+        }
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(s_full0 + 8 * b, (g >> 1) & 1, abort_flag, wlim));
         uint32_t r[HB];
         float pm = -INFINITY;
@@ -536,8 +694,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       ok = bar_and(pair_bar, 64, ok);
       if (!ok) break;
       tc_fence_after();
+      if (wr && nrow <= 0)   // an empty kept list (its partner's was not): all-zero output
+        for (int c = 0; c < HD; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
 #pragma unroll
-      for (int c = 0; c < (pad ? 0 : HD / 32); ++c) {
+      for (int c = 0; c < (pad || nrow <= 0 ? 0 : HD / 32); ++c) {
         uint32_t o[32];
         tmem_ld32(tO + c * 32, o);
         tmem_wait_ld();

@@ -46,6 +46,9 @@ CASES = {
     "single_block": _cfg("single_block", H=2, T=2, Y=8, X=8, seed=8),
     # Hilbert numbering of a 3 x 3 x 5 tile grid (non-power-of-two sides)
     "d128_hilbert": _cfg("d128_hilbert", B=1, H=4, T=6, Y=24, X=40, seed=9),
+    # 64-token tiles, an odd number of blocks per head (the last block has no partner)
+    "d64_s64_odd": _cfg("d64_s64_odd", H=3, d=64, T=5, Y=8, X=8, tt=1, ty=8, tx=8, seed=10),
+    "d128_s64_odd": _cfg("d128_s64_odd", B=2, H=2, T=3, Y=16, X=24, tt=1, ty=8, tx=8, seed=11),
 }
 HILBERT = {"d128_hilbert"}
 
@@ -310,6 +313,47 @@ def test_attention_handcrafted_lists(fva):
         for i in range(Nb):
             if not nz[0, h, i]:
                 assert (got[0, h, i * og.S:(i + 1) * og.S] == 0).all()
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_attention_handcrafted_lists_64_token_tiles(fva, d):
+    """64-token tiles run adjacent query blocks in pairs over the union of their lists:
+    empty lists on either side of a pair, full lists, unsorted ids and an odd last block
+    must each give that block's own result (zeros for an empty list)."""
+    cfg = CASES["d128_s64_odd"].with_(B=1, H=2, d=d, T=5, Y=8, X=24)   # 15 blocks per head
+    g = fva.Geom.of(cfg)
+    og = O.Geometry.of(cfg)
+    q, k, v = synth.make_qkv(cfg)
+    qr, kr, vr = (O.reorder(t, og) for t in (q, k, v))
+    rng = np.random.default_rng(3)
+    Nb = og.Nb
+    counts = rng.integers(1, Nb + 1, size=(1, 2, Nb)).astype(np.int32)
+    counts[0, 0, 0] = 0            # empty list, partner non-empty
+    counts[0, 0, 3] = 0            # partner of block 2 empty
+    counts[0, 1, 4] = 0
+    counts[0, 1, 5] = 0            # both blocks of a pair empty
+    counts[0, 1, 6] = Nb           # every block
+    counts[0, 0, Nb - 1] = 2       # the unpaired last block
+    idx = np.full((1, 2, Nb, Nb), -1, dtype=np.int32)
+    for h in range(2):
+        for i in range(Nb):
+            idx[0, h, i, :counts[0, h, i]] = rng.permutation(Nb)[:counts[0, h, i]]
+    for wl in (None, O.lpt_worklist(counts)):
+        out = torch.empty((1, 2, og.N, og.d), dtype=torch.bfloat16, device="cuda")
+        fva.fva_block_sparse_attn(to_dev(qr), to_dev(kr), to_dev(vr), torch.from_numpy(counts).cuda(),
+                                  torch.from_numpy(idx).cuda(), None if wl is None else torch.from_numpy(wl).cuda(),
+                                  g, 0.0, out)
+        torch.cuda.synchronize()
+        assert fva.fva_get_device_error() == 0
+        got = bf16_dev_to_f64(out)
+        items = [(0, h, i) for h in range(2) for i in range(Nb) if counts[0, h, i] > 0]
+        want = O.attention_items(qr, kr, vr, counts, idx, og.S, items)
+        for (b, h, i), o in want.items():
+            compare_attention(got[b, h, i * og.S:(i + 1) * og.S], o)
+        for h in range(2):
+            for i in range(Nb):
+                if counts[0, h, i] == 0:
+                    assert (got[0, h, i * og.S:(i + 1) * og.S] == 0).all()
 
 
 def test_attention_custom_scale(fva):
