@@ -59,7 +59,8 @@ def parse(argv=None):
     ap.add_argument("--tile-order", choices=("raster", "hilbert"), default="raster",
                     help="tile numbering: raster, or along the 3D Hilbert curve")
     ap.add_argument("--static-order", action="store_true", help="item-id order instead of the LPT work list")
-    ap.add_argument("--tile64", action="store_true", help="--report route: the layer with 1x8x8 tiles")
+    ap.add_argument("--tile64", action="store_true",
+                    help="the --config layer with 1x8x8 tiles (64-token blocks), for the headline line or --report route")
     ap.add_argument("--no-side-configs", action="store_true",
                     help="skip the stress720p and 64-token-tile keys of the headline line")
     ap.add_argument("--report", choices=["stress", "sweep", "sasa", "route"], default=None,
@@ -221,10 +222,16 @@ def cpu_cores() -> int:
         return os.cpu_count() or 1
 
 
+def arm_cfg(args):
+    """The --config layer, with 1x8x8 tiles when --tile64 is given."""
+    cfg = synth.CONFIGS[args.config]
+    return cfg.with_(name=cfg.name + "_tile64", tt=1) if args.tile64 else cfg
+
+
 def run_reference(args, rank: int, world: int):
     if rank != 0:
         return
-    cfg = synth.CONFIGS[args.config]
+    cfg = arm_cfg(args)
     qkv = synth.make_qkv(cfg)
     vals, secs = [], []
     desc = ""
@@ -273,7 +280,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    cfg = synth.CONFIGS[args.config]
+    cfg = arm_cfg(args)
     g = fva.Geom.of(cfg)
     if args.tile_order == "hilbert":
         g = g.with_tiles(fva.FVA_TILES_HILBERT, device=dev)

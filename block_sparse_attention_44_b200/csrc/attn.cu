@@ -46,7 +46,7 @@ constexpr int kCtrlRegs = 80;
 constexpr int kSoftmaxRegs = 192;
 // Bitmap words of one kept list (one bit per key block, up to kMaxNb blocks).
 constexpr int kBmWords = kMaxNb / 32;
-// Warps that copy the pair bitmaps (all but the K producer, which builds them).
+// Warps that copy each published work item (all but the K producer, which publishes it).
 constexpr int kBmReaders = kAttnThreads / 32 - 1;
 
 template <int D, int BN, int NSK, int NSV>
@@ -64,13 +64,13 @@ struct AttnCfg {
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
   static constexpr int OFF_V = OFF_K + NSK * KV_BYTES;
   static constexpr int OFF_BAR = OFF_V + NSV * KV_BYTES;
-  // barriers: q_full q_empty s_full[2] s_free[2] p_full[2] o_done[2] o_free drain_s drain_pv bm_full
-  // bm_empty; k ring; v ring
+  // barriers: q_full q_empty s_full[2] s_free[2] p_full[2] o_done[2] o_free drain_s drain_pv wk_full
+  // wk_empty; k ring; v ring
   static constexpr int NBAR = 15 + 2 * NSK + 2 * NSV;
   static constexpr int OFF_RED = OFF_BAR + NBAR * 8;         // row maxima / sums [2 parity][2 half][128]
   static constexpr int OFF_MISC = OFF_RED + 2 * 2 * kBM * 4; // tmem base slot, abort flag
-  static constexpr int OFF_BM = OFF_MISC + 16;               // kept-block bitmaps of a query-block pair
-  static constexpr int SMEM = OFF_BM + 2 * kBmWords * 4;     // base must be 1024-aligned (checked)
+  static constexpr int OFF_SLOT = OFF_MISC + 16;             // the work-item slot (Slot)
+  static constexpr int SMEM = OFF_SLOT + (16 + 2 * kBmWords * 4);   // base must be 1024-aligned (checked)
   // TMEM columns: S double buffer [0, 2*KN), P double buffer [2*KN, 3*KN) as bf16 pairs
   // (KN/2 columns each), O after it
   static constexpr int T_S = 0, T_P = 2 * KN, T_O = 3 * KN;
@@ -89,6 +89,8 @@ struct AttnParams {
   uint16_t* out;
   int* dev_err;
   long long n_items;
+  long long n_iter;       // work positions: list entries, or (b, h, pair) without a list
+  unsigned long long* claim;   // position counter, zero at launch; nullptr: positions at a grid stride
   int N;
   int Nb;
   float scale_log2;
@@ -135,8 +137,8 @@ __device__ __forceinline__ int item_count(const AttnParams& prm, int item) {
 // tiles: two adjacent query blocks 2p and 2p + 1 of a head share the 128-row query tile (rows
 // 0-63 and 64-127) and run over the union of their kept lists, two key blocks per S product;
 // each row masks the keys outside its own block's list, so every row's result is that of
-// its own list.  The work list's entries for odd blocks are skipped (their pair is processed
-// at the entry of the even block).
+// its own list.  The work list's entries for odd blocks carry no work (their pair runs at
+// the entry of the even block); without a list the positions are the pairs themselves.
 struct Work {
   int item;     // item id of the (first) query block
   int nq;       // query blocks in the tile (2 for a full pair)
@@ -144,7 +146,14 @@ struct Work {
 };
 template <int KPU>
 __device__ __forceinline__ bool work_at(const AttnParams& prm, long long it, Work& w) {
-  const int item = item_at(prm, it);
+  int item;
+  if (KPU == 2 && !prm.worklist) {   // position it = pair p of (b, h): item of block 2p
+    const int np = (prm.Nb + 1) / 2;
+    const long long bh = it / np;
+    item = static_cast<int>(bh * prm.Nb + 2 * (it - bh * np));
+  } else {
+    item = item_at(prm, it);
+  }
   if (item < 0) return false;
   w.item = item;
   w.n0 = item_count(prm, item);
@@ -193,9 +202,6 @@ __device__ __forceinline__ bool in_list(const Bitmaps& b, int which, int j) {
   const uint32_t lo = which ? b.b0 : b.a0, hi = which ? b.b1 : b.a1;
   return (__shfl_sync(0xffffffffu, w < 32 ? lo : hi, w & 31) >> (j & 31)) & 1u;
 }
-// Units (S products) of a work item: its kept blocks with 128-token tiles; half the union
-// of the two lists, rounded up, with 64-token tiles.
-__device__ __forceinline__ int unit_count(int n, int kpu) { return n <= 0 ? 0 : (n + kpu - 1) / kpu; }
 // Kept key block jj of item `item` (row i), replaced by the diagonal if out of range.
 __device__ __forceinline__ int block_id(const AttnParams& prm, int item, int i, int jj, bool report) {
   int j = prm.idx[static_cast<long long>(item) * prm.Nb + jj];
@@ -206,15 +212,60 @@ __device__ __forceinline__ int block_id(const AttnParams& prm, int item, int i, 
   return j;
 }
 
-// Bitmaps of a work item for the warps that read them: the K producer builds them (below);
-// every other warp waits for them, copies its lanes' words and releases the buffer.
-__device__ __forceinline__ bool copy_bitmaps(const uint32_t* bm, uint32_t bm_full, uint32_t bm_empty, long long k,
-                                             volatile int* abort_flag, long long wlim, Bitmaps& out) {
-  if (!__all_sync(0xffffffffu, mbar_wait(bm_full, k & 1, abort_flag, wlim))) return false;
-  out = load_bitmaps(bm);
+// The work-item slot in shared memory.  The K producer claims every work item and publishes
+// it here (item id, or -1 when no work is left; query blocks; list lengths; with 64-token
+// tiles the two lists' bitmaps); each of the other warps waits for it, copies it and releases
+// the slot, so all roles take the same items in the same order.
+struct Slot {
+  int item, nq, n0, n1;
+  uint32_t bm[2 * kBmWords];
+};
+static_assert(sizeof(Slot) == 16 + 2 * kBmWords * 4, "slot layout");
+template <int KPU>
+__device__ __forceinline__ bool read_work(const Slot* slot, uint32_t full, uint32_t empty, long long k,
+                                          volatile int* abort_flag, long long wlim, Work& w, Bitmaps& b) {
+  if (!__all_sync(0xffffffffu, mbar_wait(full, k & 1, abort_flag, wlim))) return false;
+  w.item = slot->item;
+  w.nq = slot->nq;
+  w.n0 = slot->n0;
+  w.n1 = slot->n1;
+  if (KPU == 2 && w.item >= 0) b = load_bitmaps(slot->bm);
   __syncwarp();
-  if ((threadIdx.x & 31) == 0) mbar_arrive(bm_empty);
+  if ((threadIdx.x & 31) == 0) mbar_arrive(empty);
   return true;
+}
+// The next work item of this CTA (whole warp, warp-uniform).  Positions are claimed from the
+// launch's counter: every CTA moves through the list with the others (the K and V blocks they
+// read at a time overlap in L2), and a CTA that finishes early takes the next item (greedy
+// list order).  Without a counter the positions come at a stride of the grid.  Positions that
+// carry no work (the odd block of a pair, an id outside the items) are passed over.
+template <int KPU>
+__device__ __forceinline__ bool next_work(const AttnParams& prm, long long& pos, Work& w) {
+  while (true) {
+    long long it;
+    if (prm.claim) {
+      unsigned long long c = 0;
+      if ((threadIdx.x & 31) == 0) c = atomicAdd(prm.claim, 1ull);
+      it = static_cast<long long>(__shfl_sync(0xffffffffu, c, 0));
+    } else {
+      it = pos < 0 ? static_cast<long long>(blockIdx.x) : pos + gridDim.x;
+      pos = it;
+    }
+    if (it >= prm.n_iter) return false;
+    if (work_at<KPU>(prm, it, w)) return true;
+  }
+}
+// The next work item of a warp other than the K producer: 1 (w and, with 64-token tiles, b
+// filled), 0 when no work is left, -1 when the wait expired.  With 128-token tiles every warp
+// takes the positions at the grid stride itself (no claims, no slot: measured faster there,
+// where every position carries work); with 64-token tiles it reads the published item.
+template <int KPU>
+__device__ __forceinline__ int take_work(const AttnParams& prm, long long& pos, const Slot* slot, uint32_t full,
+                                         uint32_t empty, long long& pubs, volatile int* abort_flag, long long wlim,
+                                         Work& w, Bitmaps& b) {
+  if (KPU == 1) return next_work<1>(prm, pos, w) ? 1 : 0;
+  if (!read_work<KPU>(slot, full, empty, pubs++, abort_flag, wlim, w, b)) return -1;
+  return w.item < 0 ? 0 : 1;
 }
 
 // One TMA producer warp: one ring stage (K or V, 64-column boxes) per unit of KPU key blocks
@@ -226,46 +277,61 @@ __device__ __forceinline__ bool copy_bitmaps(const uint32_t* bm, uint32_t bm_ful
 template <int D, int BN, int NS, bool WITH_Q, typename Cfg>
 __device__ void produce(const AttnParams& prm, const CUtensorMap* tm, const CUtensorMap* tmQ, uint32_t ring,
                         uint32_t full0, uint32_t empty0, uint32_t sQ, uint32_t q_full, uint32_t q_empty,
-                        uint32_t* bm, uint32_t bm_full, uint32_t bm_empty, volatile int* abort_flag) {
+                        Slot* slot, uint32_t wk_full, uint32_t wk_empty, volatile int* abort_flag) {
   const int Nb = prm.Nb;
   const int lane = threadIdx.x & 31;
   const bool leader = lane == 0;
   const int nwords = (Nb + 31) / 32;
-  long long g = 0, q_items = 0, pairs = 0;
+  long long g = 0, q_items = 0, pubs = 0, pos = -1;
   bool ok = true;
-  for (long long it = blockIdx.x; it < prm.n_items && ok; it += gridDim.x) {
-    Work w;
-    if (!work_at<Cfg::KPU>(prm, it, w) || w.n0 + w.n1 <= 0) continue;
-    const long long bh = w.item / Nb;
-    const int i = w.item - static_cast<int>(bh * Nb);
-    const long long row0 = bh * prm.N;
+  while (ok) {
+    Work w{-1, 0, 0, 0};
     Bitmaps bmr{0, 0, 0, 0};
-    int nu = w.n0;
-    if (Cfg::KPU == 2) {
-      if (WITH_Q) {
-        // every reader has copied the previous pair's bitmaps
-        if (pairs > 0 &&
-            !(ok = __all_sync(0xffffffffu, mbar_wait(bm_empty, (pairs - 1) & 1, abort_flag, prm.wait_limit))))
-          break;
-        for (int e = lane; e < 2 * kBmWords; e += 32) bm[e] = 0u;
+    if (WITH_Q && Cfg::KPU == 1) {
+      if (!next_work<1>(prm, pos, w)) break;
+    } else if (WITH_Q) {
+      // claim the next item, then publish it once every reader has copied the previous one
+      const bool have = next_work<Cfg::KPU>(prm, pos, w);
+      if (pubs > 0 &&
+          !(ok = __all_sync(0xffffffffu, mbar_wait(wk_empty, (pubs - 1) & 1, abort_flag, prm.wait_limit))))
+        break;
+      if (!have) w.item = -1;
+      if (Cfg::KPU == 2 && have && w.n0 + w.n1 > 0) {
+        const int i = w.item % Nb;
+        for (int e = lane; e < 2 * kBmWords; e += 32) slot->bm[e] = 0u;
         __syncwarp();
         for (int x = 0; x < w.nq; ++x) {
           const int n = x ? w.n1 : w.n0;
           for (int c = lane; c < n; c += 32) {
             const int j = block_id(prm, w.item + x, i + x, c, true);
-            atomicOr(&bm[x * kBmWords + (j >> 5)], 1u << (j & 31));
+            atomicOr(&slot->bm[x * kBmWords + (j >> 5)], 1u << (j & 31));
           }
         }
-        __threadfence_block();
-        __syncwarp();
-        if (leader) mbar_arrive(bm_full);
-        bmr = load_bitmaps(bm);
-      } else if (!(ok = copy_bitmaps(bm, bm_full, bm_empty, pairs, abort_flag, prm.wait_limit, bmr))) {
+      }
+      if (leader) {
+        slot->item = w.item;
+        slot->nq = w.nq;
+        slot->n0 = w.n0;
+        slot->n1 = w.n1;
+      }
+      __threadfence_block();
+      __syncwarp();
+      if (leader) mbar_arrive(wk_full);
+      ++pubs;
+      if (!have) break;
+      if (Cfg::KPU == 2 && w.n0 + w.n1 > 0) bmr = load_bitmaps(slot->bm);
+    } else {
+      const int t = take_work<Cfg::KPU>(prm, pos, slot, wk_full, wk_empty, pubs, abort_flag, prm.wait_limit, w, bmr);
+      if (t <= 0) {
+        ok = t == 0;
         break;
       }
-      ++pairs;
-      nu = (union_size(bmr) + 1) / 2;
     }
+    if (w.n0 + w.n1 <= 0) continue;   // an empty list: nothing to load (the softmax writes zeros)
+    const long long bh = w.item / Nb;
+    const int i = w.item - static_cast<int>(bh * Nb);
+    const long long row0 = bh * prm.N;
+    const int nu = Cfg::KPU == 2 ? (union_size(bmr) + 1) / 2 : w.n0;
     if (WITH_Q) {
       if (q_items > 0 &&
           !(ok = __all_sync(0xffffffffu, mbar_wait(q_empty, (q_items - 1) & 1, abort_flag, prm.wait_limit))))
@@ -335,14 +401,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t bar0 = sbase + C::OFF_BAR;
   const uint32_t q_full = bar0, q_empty = bar0 + 8, s_full0 = bar0 + 16, s_free0 = bar0 + 32;
   const uint32_t p_full0 = bar0 + 48, o_done0 = bar0 + 64, o_free = bar0 + 80, drain_s = bar0 + 88;
-  const uint32_t drain_pv = bar0 + 96, bm_full = bar0 + 104, bm_empty = bar0 + 112;
+  const uint32_t drain_pv = bar0 + 96, wk_full = bar0 + 104, wk_empty = bar0 + 112;
   const uint32_t k_full0 = bar0 + 120;
   const uint32_t k_empty0 = k_full0 + 8 * NSK;
   const uint32_t v_full0 = k_empty0 + 8 * NSK;
   const uint32_t v_empty0 = v_full0 + 8 * NSV;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
-  uint32_t* bm = reinterpret_cast<uint32_t*>(smem + C::OFF_BM);
+  Slot* slot = reinterpret_cast<Slot*>(smem + C::OFF_SLOT);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x & 31;
@@ -359,8 +425,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     mbar_init(o_free, 256);
     mbar_init(drain_s, 1);
     mbar_init(drain_pv, 1);
-    mbar_init(bm_full, 1);
-    mbar_init(bm_empty, kBmReaders);
+    mbar_init(wk_full, 1);
+    mbar_init(wk_empty, kBmReaders);
     for (int st = 0; st < NSK; ++st) {
       mbar_init(k_full0 + 8 * st, 1);
       mbar_init(k_empty0 + 8 * st, 1);
@@ -394,7 +460,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  const long long n_items = prm.n_items;
   const int Nb = prm.Nb;
   const int S = BN;
   const bool leader = lane == 0;
@@ -411,11 +476,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtrlRegs));
   if (warp == 0) {
     // ---------------------------------------------------------------- Q + K producer
-    produce<D, BN, NSK, true, C>(prm, &tmK, &tmQ, sK, k_full0, k_empty0, sQ, q_full, q_empty, bm, bm_full, bm_empty,
+    produce<D, BN, NSK, true, C>(prm, &tmK, &tmQ, sK, k_full0, k_empty0, sQ, q_full, q_empty, slot, wk_full, wk_empty,
                                  abort_flag);
   } else if (warp == 3) {
     // ---------------------------------------------------------------- V producer
-    produce<D, BN, NSV, false, C>(prm, &tmV, &tmQ, sV, v_full0, v_empty0, sQ, q_full, q_empty, bm, bm_full, bm_empty,
+    produce<D, BN, NSV, false, C>(prm, &tmV, &tmQ, sV, v_full0, v_empty0, sQ, q_full, q_empty, slot, wk_full, wk_empty,
                                   abort_flag);
   } else if (warp == 1) {
     // ---------------------------------------------------------------- S issuer
@@ -428,19 +493,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint64_t dK0 = sdesc_sw128(sK, 16, 1024);
     // (descriptor start addresses are the low 14 bits, address >> 4; operands lie
     //  below 256 KB, so byte offsets add in without carry)
-    long long g = 0, q_items = 0, pairs = 0;
+    long long g = 0, q_items = 0, pubs = 0, pos = -1;
     bool ok = true, issued = false;
-    for (long long it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-      Work w;
-      if (!work_at<C::KPU>(prm, it, w) || w.n0 + w.n1 <= 0) continue;
+    while (ok) {
+      Work w{-1, 0, 0, 0};
+      Bitmaps bmr{0, 0, 0, 0};
+      const int t = take_work<C::KPU>(prm, pos, slot, wk_full, wk_empty, pubs, abort_flag, wlim, w, bmr);
+      if (t <= 0) {
+        ok = t == 0;
+        break;
+      }
+      if (w.n0 + w.n1 <= 0) continue;
       if (!(ok = wait_all(q_full, q_items & 1))) break;
       ++q_items;
-      int nu = w.n0;
-      if (C::KPU == 2) {
-        Bitmaps bmr;
-        if (!(ok = copy_bitmaps(bm, bm_full, bm_empty, pairs++, abort_flag, wlim, bmr))) break;
-        nu = (union_size(bmr) + 1) / 2;
-      }
+      const int nu = C::KPU == 2 ? (union_size(bmr) + 1) / 2 : w.n0;
       for (int jj = 0; jj < nu; ++jj, ++g) {
         const int b = static_cast<int>(g & 1);
         const int st = static_cast<int>(g % NSK);
@@ -478,17 +544,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // O += P_j V_j once the softmax has written P_j into P buffer j % 2 (p_full); the
     // commit on o_done[j % 2] tells the softmax that buffer and O are free again.
     const uint64_t dV0 = sdesc_sw128(sV, C::KV_CHUNK, 1024);
-    long long g = 0, items = 0, pairs = 0;
+    long long g = 0, items = 0, pubs = 0, pos = -1;
     bool ok = true, issued = false;
-    for (long long it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-      Work w;
-      if (!work_at<C::KPU>(prm, it, w) || w.n0 + w.n1 <= 0) continue;
-      int nu = w.n0;
-      if (C::KPU == 2) {
-        Bitmaps bmr;
-        if (!(ok = copy_bitmaps(bm, bm_full, bm_empty, pairs++, abort_flag, wlim, bmr))) break;
-        nu = (union_size(bmr) + 1) / 2;
+    while (ok) {
+      Work w{-1, 0, 0, 0};
+      Bitmaps bmr{0, 0, 0, 0};
+      const int t = take_work<C::KPU>(prm, pos, slot, wk_full, wk_empty, pubs, abort_flag, wlim, w, bmr);
+      if (t <= 0) {
+        ok = t == 0;
+        break;
       }
+      if (w.n0 + w.n1 <= 0) continue;
+      const int nu = C::KPU == 2 ? (union_size(bmr) + 1) / 2 : w.n0;
       if (items > 0 && !(ok = wait_all(o_free, (items - 1) & 1))) break;   // epilogue read O
       for (int jj = 0; jj < nu; ++jj, ++g) {
         const int st = static_cast<int>(g % NSV);
@@ -543,7 +610,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     float* red_max = reinterpret_cast<float*>(smem + C::OFF_RED);         // [2][2][kBM]
     const float sl2 = prm.scale_log2;
     const uint64_t sl2x2 = f32x2_pack(sl2, sl2);
-    long long g = 0, pairs = 0;   // units processed; pairs whose bitmaps were copied
+    long long g = 0, pubs = 0, pos = -1;   // units processed; work items read; list position
     bool ok = true;
     // wait until P_q V_q has completed (its commit on o_done[q % 2] is that barrier's
     // phase q / 2; P_{q+2} V_{q+2} cannot start before this warp writes P_{q+2}, so the
@@ -553,9 +620,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         ok = __all_sync(0xffffffffu, mbar_wait(o_done0 + 8 * static_cast<uint32_t>(q & 1), (q >> 1) & 1, abort_flag,
                                                wlim));
     };
-    for (long long it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-      Work w;
-      if (!work_at<C::KPU>(prm, it, w)) continue;
+    while (ok) {
+      Work w{-1, 0, 0, 0};
+      Bitmaps bmr{0, 0, 0, 0};
+      const int t = take_work<C::KPU>(prm, pos, slot, wk_full, wk_empty, pubs, abort_flag, wlim, w, bmr);
+      if (C::KPU == 2) {
+        // both warps of the quarter leave together or not at all: a warp whose wait expired
+        // still meets its partner here, so neither is left waiting at a pair barrier
+        ok = bar_and(pair_bar, 64, t >= 0);
+        if (!ok) break;
+      }
+      if (t <= 0) break;
       const long long bh = w.item / Nb;
       const int i = w.item - static_cast<int>(bh * Nb);
       // rows of a query block the tile does not hold (64-token tiles: the odd last block of a
@@ -572,12 +647,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           for (int c = 0; c < HD; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
         continue;
       }
-      Bitmaps bmr{0, 0, 0, 0};
-      int nu = w.n0;
-      if (C::KPU == 2) {
-        if (!(ok = copy_bitmaps(bm, bm_full, bm_empty, pairs++, abort_flag, wlim, bmr))) break;
-        nu = (union_size(bmr) + 1) / 2;
-      }
+      const int nu = C::KPU == 2 ? (union_size(bmr) + 1) / 2 : w.n0;
       Cursor cur;
       float m = -INFINITY;   // running max of the scaled logits (base-2 units), same in both halves
       float l = 0.0f;        // this half's running row sum at max m
@@ -784,7 +854,7 @@ cudaError_t launch_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
   cudaError_t e =
       cudaFuncSetAttribute(attn_kernel<D, BN, NSK, NSV>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  const long long grid = prm.n_items < sm_count() ? prm.n_items : sm_count();
+  const long long grid = prm.n_iter < sm_count() ? prm.n_iter : sm_count();
   attn_kernel<D, BN, NSK, NSV><<<static_cast<unsigned>(grid), kAttnThreads, C::SMEM, s>>>(mq, mk, mv, prm);
   return cudaGetLastError();
 }
@@ -795,7 +865,8 @@ void set_attn_wait_limit(long long cycles) { g_wait_limit.store(cycles > 0 ? cyc
 
 cudaError_t launch_attention(const void* qr, const void* kr, const void* vr, const int32_t* counts, const int32_t* idx,
                              const int32_t* worklist, const Dims& D, const fva_geom* natural, float scale, void* out,
-                             int* dev_err, cudaStream_t s, int* launches, char* msg, size_t msg_len) {
+                             int* dev_err, unsigned long long* claim, cudaStream_t s, int* launches, char* msg,
+                             size_t msg_len) {
   const long long rows = D.BH() * D.N;
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, qr, rows, D.d, D.S, msg, msg_len) || !make_map(&mk, kr, rows, D.d, D.S, msg, msg_len) ||
@@ -808,6 +879,10 @@ cudaError_t launch_attention(const void* qr, const void* kr, const void* vr, con
   prm.out = static_cast<uint16_t*>(out);
   prm.dev_err = dev_err;
   prm.n_items = D.rows();
+  // 64-token tiles run pairs of query blocks: without a work list the positions are the
+  // pairs themselves, with one the entries of odd blocks carry no work
+  prm.n_iter = (D.S < 128 && !worklist) ? D.BH() * ((D.Nb + 1) / 2) : D.rows();
+  prm.claim = D.S < 128 ? claim : nullptr;   // claims only for 64-token pairs
   prm.N = D.N;
   prm.Nb = D.Nb;
   prm.scale_log2 = scale * 1.4426950408889634f;
@@ -823,6 +898,7 @@ cudaError_t launch_attention(const void* qr, const void* kr, const void* vr, con
   const long long wl = g_wait_limit.load();
   prm.wait_limit = wl > 0 ? wl : kWaitLimitCycles;
   cudaError_t e;
+  if (prm.claim && (e = cudaMemsetAsync(prm.claim, 0, sizeof(*prm.claim), s)) != cudaSuccess) return e;
   if (D.d == 128 && D.S == 128)
     e = launch_t<128, 128, 3, 3>(mq, mk, mv, prm, s);
   else if (D.d == 128 && D.S == 64)

@@ -24,6 +24,9 @@ std::atomic<long long> g_launches{0};
 // fva_get_device_error(stream) reads and clears that word only.
 constexpr int kErrSlots = 64;
 __device__ int g_dev_err[kErrSlots];
+// Work-claim counters of the attention kernel, one per stream slot like the error words; a
+// stream on the shared slot 0 gets none (two launches in flight must not share a counter).
+__device__ unsigned long long g_claim[kErrSlots];
 
 int fail(int code, const char* fmt, ...) {
   va_list ap;
@@ -37,26 +40,59 @@ int cuda_fail(cudaError_t e, const char* where) {
   return fail(FVA_ERR_CUDA, "%s: %s (%s)", where, cudaGetErrorName(e), cudaGetErrorString(e));
 }
 
-// Error word of `stream` on the current device (nullptr if the runtime cannot say).
-int* dev_err_ptr(void* stream) {
+// Slot of `stream` on the current device (1 .. kErrSlots - 1 for the first streams seen, 0 for
+// any further stream) and the device's base addresses of the error words and claim counters;
+// false if the runtime cannot say.
+bool stream_slot(void* stream, int** err_base, unsigned long long** claim_base, int* slot_out) {
   constexpr int kMaxDev = 64;
   static std::mutex mu;
-  static int* base[kMaxDev] = {nullptr};                 // the array's address differs per device
+  static int* ebase[kMaxDev] = {nullptr};                // the arrays' addresses differ per device
+  static unsigned long long* cbase[kMaxDev] = {nullptr};
   static std::vector<std::pair<void*, int>> slots[kMaxDev];
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return nullptr;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return false;
   std::lock_guard<std::mutex> lock(mu);
-  if (!base[dev]) {
+  if (!ebase[dev]) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_dev_err) != cudaSuccess) return nullptr;
-    base[dev] = static_cast<int*>(p);
+    void* c = nullptr;
+    if (cudaGetSymbolAddress(&p, g_dev_err) != cudaSuccess || cudaGetSymbolAddress(&c, g_claim) != cudaSuccess)
+      return false;
+    ebase[dev] = static_cast<int*>(p);
+    cbase[dev] = static_cast<unsigned long long*>(c);
   }
+  *err_base = ebase[dev];
+  *claim_base = cbase[dev];
   for (const auto& e : slots[dev])
-    if (e.first == stream) return base[dev] + e.second;
+    if (e.first == stream) {
+      *slot_out = e.second;
+      return true;
+    }
   const int slot = static_cast<int>(slots[dev].size()) + 1;
-  if (slot >= kErrSlots) return base[dev];                // table full: the shared word
+  if (slot >= kErrSlots) {                               // table full: the shared word
+    *slot_out = 0;
+    return true;
+  }
   slots[dev].emplace_back(stream, slot);
-  return base[dev] + slot;
+  *slot_out = slot;
+  return true;
+}
+
+// Error word of `stream` on the current device (nullptr if the runtime cannot say).
+int* dev_err_ptr(void* stream) {
+  int* eb = nullptr;
+  unsigned long long* cb = nullptr;
+  int slot = 0;
+  if (!stream_slot(stream, &eb, &cb, &slot)) return nullptr;
+  return eb + slot;
+}
+
+// Work-claim counter of `stream` (nullptr on the shared slot or if the runtime cannot say).
+unsigned long long* claim_ptr(void* stream) {
+  int* eb = nullptr;
+  unsigned long long* cb = nullptr;
+  int slot = 0;
+  if (!stream_slot(stream, &eb, &cb, &slot) || slot == 0) return nullptr;
+  return cb + slot;
 }
 
 // Validates the geometry; fills D.  Returns FVA_OK or an error code (message set).
@@ -366,7 +402,8 @@ static int attn_common(const void* qr, const void* kr, const void* vr, const int
   char msg[256] = "";
   int launches = 0;
   cudaError_t e = fva::launch_attention(qr, kr, vr, counts, idx, worklist, D, natural ? &g : nullptr, scale, out, de,
-                                        static_cast<cudaStream_t>(stream), &launches, msg, sizeof(msg));
+                                        claim_ptr(stream), static_cast<cudaStream_t>(stream), &launches, msg,
+                                        sizeof(msg));
   if (msg[0]) {
     g_launches += launches;
     return fail(FVA_ERR_CUDA, "%s: %s", name, msg);

@@ -64,8 +64,11 @@ void set_attn_wait_limit(long long cycles);
 
 // Block-sparse attention (tcgen05).
 // natural != nullptr: O is written in natural token order of that geometry.
+// claim: a device counter private to this stream (zeroed here before the launch) from which
+// the CTAs claim work positions, or nullptr for positions at a grid stride.
 cudaError_t launch_attention(const void* qr, const void* kr, const void* vr, const int32_t* counts, const int32_t* idx,
                              const int32_t* worklist, const Dims& D, const fva_geom* natural, float scale, void* out,
-                             int* dev_err, cudaStream_t s, int* launches, char* msg, size_t msg_len);
+                             int* dev_err, unsigned long long* claim, cudaStream_t s, int* launches, char* msg,
+                             size_t msg_len);
 
 }  // namespace fva

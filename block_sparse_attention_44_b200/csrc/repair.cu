@@ -102,12 +102,24 @@ __global__ void __launch_bounds__(kLptThreads) lpt_hist_kernel(const int32_t* __
 
 // One CTA.  Thread-owned values v: total[v] = sum over chunks; base[v] = number of items
 // with a larger count (block scan over v descending); then hist[c][v] is replaced by
-// base[v] + sum of hist[c'][v] over chunks c' < c.
+// base[v] + sum of hist[c'][v] over chunks c' < c.  STAGED: the histograms are first
+// copied into shared memory in one coalesced pass, so the two passes over the chunks read
+// shared memory instead of waiting on dependent rounds of global loads.
+template <bool STAGED>
 __global__ void __launch_bounds__(kLptScanThreads) lpt_offsets_kernel(int32_t* __restrict__ hist, long long BH,
                                                                       int Nb) {
   constexpr int VPT = (kMaxNb + 1 + kLptScanThreads - 1) / kLptScanThreads;   // values per thread
   __shared__ long long warp_tot[kLptScanThreads / 32];
+  extern __shared__ int32_t staged[];
   const int V = Nb + 1;
+  const int32_t* src = hist;
+  if (STAGED) {
+    const long long n = BH * V;
+#pragma unroll 8
+    for (long long e = threadIdx.x; e < n; e += kLptScanThreads) staged[e] = hist[e];
+    __syncthreads();
+    src = staged;
+  }
   // thread t owns the values v = V - 1 - (t * VPT + e), e < VPT: descending order runs
   // with the thread index, so an exclusive scan over threads gives "larger counts first"
   long long tot[VPT];
@@ -119,7 +131,7 @@ __global__ void __launch_bounds__(kLptScanThreads) lpt_offsets_kernel(int32_t* _
     if (r < V) {
       const int v = V - 1 - r;
 #pragma unroll 8
-      for (long long c = 0; c < BH; ++c) tot[e] += hist[c * V + v];
+      for (long long c = 0; c < BH; ++c) tot[e] += src[c * V + v];
     }
     mine += tot[e];
   }
@@ -144,7 +156,7 @@ __global__ void __launch_bounds__(kLptScanThreads) lpt_offsets_kernel(int32_t* _
       long long run = base;
 #pragma unroll 8
       for (long long c = 0; c < BH; ++c) {
-        const int n = hist[c * V + v];
+        const int n = src[c * V + v];
         hist[c * V + v] = static_cast<int32_t>(run);
         run += n;
       }
@@ -194,7 +206,16 @@ cudaError_t launch_lpt(const int32_t* counts, const Dims& D, int64_t* head_work,
   ++*launches;
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  lpt_offsets_kernel<<<1, kLptScanThreads, 0, s>>>(hist, D.BH(), D.Nb);
+  // histograms staged in shared memory when they fit (up to 227 KB less the kernel's static share)
+  const size_t staged = static_cast<size_t>(D.BH()) * (D.Nb + 1) * sizeof(int32_t);
+  if (staged <= 232448 - 1024) {
+    e = cudaFuncSetAttribute(lpt_offsets_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(staged));
+    if (e != cudaSuccess) return e;
+    lpt_offsets_kernel<true><<<1, kLptScanThreads, staged, s>>>(hist, D.BH(), D.Nb);
+  } else {
+    lpt_offsets_kernel<false><<<1, kLptScanThreads, 0, s>>>(hist, D.BH(), D.Nb);
+  }
   ++*launches;
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   lpt_scatter_kernel<<<grid, 32, hsmem + static_cast<size_t>(D.Nb) * sizeof(int), s>>>(counts, D.Nb, hist, worklist);

@@ -250,6 +250,14 @@ int fva_repair(const uint8_t* topp_mask, const int32_t* topk_idx, fva_geom g, in
  *                over the union J of the kept key blocks of query block i.
  * tcgen05 tensor-core MMAs (bf16 in, fp32 accumulate in TMEM), fp32 online softmax,
  * bf16 round-to-nearest output.  Requires d in {64, 128} and S = tt*ty*tx in {64, 128}.
+ * Scheduling: one persistent CTA per SM.  S = 128: CTA c takes list positions c, c + grid,
+ * c + 2 grid, ...  S = 64: adjacent query blocks 2p, 2p+1 of a head run as one item over the
+ * union of their lists (each row still sees only its own list); the list's entries for odd
+ * blocks carry no work, and each CTA claims the next position from a counter private to
+ * `stream` (an 8-byte memset on `stream` precedes the kernel), so free CTAs take items in
+ * list order (greedy) and all CTAs work through nearby positions at a time.  A process's
+ * 64th and later streams on a device share one error word and get no counter: their
+ * positions come at the grid stride instead (same results).
  */
 int fva_block_sparse_attn(const void* qr, const void* kr, const void* vr,
                           const int32_t* counts, const int32_t* idx, const int32_t* worklist,
