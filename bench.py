@@ -100,9 +100,15 @@ def load_peaks() -> dict:
 
 
 def attn_source_hash() -> str:
+    """Hash of the attention kernel's code (attn.cu + fva_common.cuh) with // comments and
+    blank lines removed, so that only a change of the code itself invalidates a capture."""
     h = hashlib.sha256()
     for f in ("attn.cu", "fva_common.cuh"):
-        h.update(open(os.path.join(ROOT, "block_sparse_attention_44_b200", "csrc", f), "rb").read())
+        text = open(os.path.join(ROOT, "block_sparse_attention_44_b200", "csrc", f), encoding="utf-8").read()
+        for line in text.splitlines():
+            code = re.sub(r"//.*$", "", line).rstrip()
+            if code:
+                h.update(code.encode() + b"\n")
     return h.hexdigest()[:12]
 
 

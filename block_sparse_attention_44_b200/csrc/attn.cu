@@ -4,11 +4,13 @@
 // query/key block pairs are evaluated).
 //
 // Persistent kernel, one CTA per SM, walking a work list of (b, h, query-block)
-// items (heavy items first when the caller passes the LPT list).  Per item the CTA
-// keeps the 128-row Q tile in shared memory and streams the item's kept K and V
-// blocks through two TMA rings; a K stage is released as soon as its S product is
-// done, a V stage after its PV product.  Roles (12 warps):
-//   warp 0    : TMA producer  — Q once per item, K_j per kept block
+// items (heavy items first when the caller passes the LPT list): with 128-token tiles at
+// a stride of the grid, with 64-token tiles (two query blocks per item) by claiming list
+// positions from a counter.  Per item the CTA keeps the 128-row Q tile in shared memory
+// and streams the item's kept K and V blocks through two TMA rings; a K stage is released
+// as soon as its S product is done, a V stage after its PV product.  Roles (12 warps):
+//   warp 0    : TMA producer  — Q once per item, K_j per kept block; with 64-token tiles
+//               it also claims each item and publishes it to the other warps
 //   warp 3    : TMA producer  — V_j per kept block
 //   warp 1    : MMA issuer    — S_j = Q K_j^T (both operands in shared memory)
 //   warp 2    : MMA issuer    — O += P_j V_j (P from tensor memory); allocates TMEM
