@@ -356,6 +356,73 @@ def test_attention_handcrafted_lists_64_token_tiles(fva, d):
                     assert (got[0, h, i * og.S:(i + 1) * og.S] == 0).all()
 
 
+def _pairs_on_claimless_stream():
+    """Body of test_64_token_pairs_on_a_stream_without_claim_counter, run in a child process:
+    it fills that process's table of per-stream slots, which later tests of this process rely
+    on being free."""
+    import block_sparse_attention_44_b200 as fva
+    from cuda.bindings import runtime as rt
+    cfg = CASES["d128_s64_odd"].with_(B=1, H=2, T=5, Y=8, X=24)   # 15 blocks per head
+    g = fva.Geom.of(cfg)
+    og = O.Geometry.of(cfg)
+    q, k, v = synth.make_qkv(cfg)
+    qr, kr, vr = (O.reorder(t, og) for t in (q, k, v))
+    rng = np.random.default_rng(5)
+    Nb = og.Nb
+    counts = rng.integers(1, Nb + 1, size=(1, 2, Nb)).astype(np.int32)
+    idx = np.full((1, 2, Nb, Nb), -1, dtype=np.int32)
+    for h in range(2):
+        for i in range(Nb):
+            idx[0, h, i, :counts[0, h, i]] = rng.permutation(Nb)[:counts[0, h, i]]
+    qd, kd, vd = to_dev(qr), to_dev(kr), to_dev(vr)
+    cd, xd = torch.from_numpy(counts).cuda(), torch.from_numpy(idx).cuda()
+    wl = torch.from_numpy(O.lpt_worklist(counts)).cuda()
+    streams = []
+    torch.cuda.synchronize()
+    try:
+        for _ in range(70):
+            err, st = rt.cudaStreamCreate()
+            assert err == rt.cudaError_t.cudaSuccess
+            streams.append(st)
+        scratch = torch.empty((1, 2, og.N, og.d), dtype=torch.bfloat16, device="cuda")
+        for st in streams:
+            fva.fva_block_sparse_attn(qd, kd, vd, cd, xd, wl, g, 0.0, scratch, stream=int(st))
+        torch.cuda.synchronize()
+        last = int(streams[-1])
+        fva.fva_get_device_error(last)   # the shared word starts clear for the checked calls
+        items = [(0, h, i) for h in range(2) for i in range(Nb)]
+        want = O.attention_items(qr, kr, vr, counts, idx, og.S, items)
+        for lst in (None, wl):
+            out = torch.empty((1, 2, og.N, og.d), dtype=torch.bfloat16, device="cuda")
+            fva.fva_block_sparse_attn(qd, kd, vd, cd, xd, lst, g, 0.0, out, stream=last)
+            torch.cuda.synchronize()
+            assert fva.fva_get_device_error(last) == 0
+            got = bf16_dev_to_f64(out)
+            for (b, h, i), o in want.items():
+                compare_attention(got[b, h, i * og.S:(i + 1) * og.S], o)
+    finally:
+        torch.cuda.synchronize()
+        for st in streams:
+            rt.cudaStreamDestroy(st)
+
+
+def test_64_token_pairs_on_a_stream_without_claim_counter(fva):
+    """A process's 64th and later streams on a device share error word 0 and get no work-claim
+    counter, so 64-token pairs there take list positions at the grid stride instead of claiming
+    them.  A child process creates seventy fresh streams (the slot table keeps at most 63 streams
+    of their own), makes one call per stream, and on the last one, with and without the LPT list,
+    every block must get its own list's result."""
+    import os
+    import subprocess
+    import sys
+    here = os.path.dirname(os.path.abspath(__file__))
+    root = os.path.dirname(here)
+    code = ("import sys; sys.path[:0] = [%r, %r]; import test_gpu_parity as t; t._pairs_on_claimless_stream()"
+            % (root, here))
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, (r.stdout[-3000:] + r.stderr[-3000:])
+
+
 def test_attention_custom_scale(fva):
     cfg = CASES["tiny"]
     g = fva.Geom.of(cfg)
