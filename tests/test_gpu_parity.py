@@ -49,8 +49,11 @@ CASES = {
     # 64-token tiles, an odd number of blocks per head (the last block has no partner)
     "d64_s64_odd": _cfg("d64_s64_odd", H=3, d=64, T=5, Y=8, X=8, tt=1, ty=8, tx=8, seed=10),
     "d128_s64_odd": _cfg("d128_s64_odd", B=2, H=2, T=3, Y=16, X=24, tt=1, ty=8, tx=8, seed=11),
+    # 64-token pairs with Hilbert numbering of a 5 x 3 x 5 tile grid (75 blocks: the last one
+    # unpaired); the natural-order epilogue places both blocks of a pair through the table
+    "d128_s64_hilbert": _cfg("d128_s64_hilbert", B=1, H=2, T=5, Y=24, X=40, tt=1, ty=8, tx=8, seed=12),
 }
-HILBERT = {"d128_hilbert"}
+HILBERT = {"d128_hilbert", "d128_s64_hilbert"}
 
 
 @pytest.mark.parametrize("name", list(CASES))
