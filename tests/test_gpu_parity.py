@@ -527,17 +527,21 @@ def test_device_error_word_is_per_stream(fva):
     assert fva.fva_get_device_error(s1) == 0
 
 
-def test_wait_expiry_reports_timeout_and_recovers(fva):
+@pytest.mark.parametrize("name,use_list", [("d128_s128_multiwave", False), ("d128_s64_odd", True)])
+def test_wait_expiry_reports_timeout_and_recovers(fva, name, use_list):
     """With the pipeline wait limit far below a copy's latency every CTA gives up: the
     call reports FVA_ERR_TIMEOUT (device word 1) after draining its copies and products,
-    and the next call with the default limit on the same stream is correct."""
-    cfg = CASES["d128_s128_multiwave"]
+    and the next call with the default limit on the same stream is correct.  The 64-token
+    case runs claimed, published work items from the LPT list, so the waits on the
+    work-item slot and the softmax warps' meeting at every item fetch give up too."""
+    cfg = CASES[name]
     g = fva.Geom.of(cfg)
     og = O.Geometry.of(cfg)
     q, k, v = synth.make_qkv(cfg)
     qr, kr, vr = (O.reorder(t, og) for t in (q, k, v))
     counts, idx = _full_lists(og)
-    args = [to_dev(qr), to_dev(kr), to_dev(vr), torch.from_numpy(counts).cuda(), torch.from_numpy(idx).cuda(), None,
+    wl = torch.from_numpy(O.lpt_worklist(counts)).cuda() if use_list else None
+    args = [to_dev(qr), to_dev(kr), to_dev(vr), torch.from_numpy(counts).cuda(), torch.from_numpy(idx).cuda(), wl,
             g, 0.0]
     out = torch.zeros((og.B, og.H, og.N, og.d), dtype=torch.bfloat16, device="cuda")
     torch.cuda.synchronize()
